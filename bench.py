@@ -1,0 +1,460 @@
+"""Benchmark of the NVFP4 training hot path on B200.
+
+One step = the three training GEMMs (fprop, dgrad, wgrad) of both linears of a 12B-class
+MLP (tokens 8192, d_model 5120, up 5120 -> 20480, down 20480 -> 5120), each with the
+quantization of its two operands: 2D-scaled weights, 1x16 activations, stochastically
+rounded gradients, random-Hadamard-transformed wgrad inputs.  Every kernel is the library's
+(libnvfp4.so through its C ABI); the timed region queues the same calls the nvfp4_linear_*
+entry points make, with CUDA events around each GEMM and each quantizer launch.
+
+Prints one JSON line (rank 0).  `--impl reference` times the CPU oracle instead, on a bounded
+sample of the same workload.  Under torchrun (N > 1) every rank runs an independent replica
+on its own GPU (the path has no exchange step); the time is the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "NVFP4 GEMM TFLOPS & quantize GB/s on 1 B200, % of FP4/HBM roofline"
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ---- multi-rank plumbing (also exercised by the CPU gloo tests) --------------------------
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank scalar over the process group (identity without one)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, seconds_max: float) -> float:
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / seconds_max
+
+
+# ---- clocks ------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.device_index = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---- the workload ------------------------------------------------------------------------
+
+OPS = ("fprop", "dgrad", "wgrad")
+
+
+class Step:
+    """Device buffers and the call sequence of one step of the MLP workload."""
+
+    def __init__(self, workload, device, seed_offset=0):
+        import torch
+        from nvfp4_bit_quantized_03_b200 import binding as B
+        self.B = B
+        self.torch = torch
+        self.wl = workload
+        self.device = device
+        self.seed = workload.seed
+        self.mask = B.sign_mask_from_seed(workload.seed)
+        self.host = []     # pinned host copies of the inputs (for the end-to-end timing)
+        self.layers = []
+        for li, lin in enumerate(workload.linears):
+            X, W, dY = synth.linear_inputs(lin, workload.seed, layer_index=li)
+            tens = {}
+            for name, arr in (("X", X), ("W", W), ("dY", dY)):
+                h = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16).pin_memory()
+                self.host.append(h)
+                tens[name] = h.to(device)
+            T, I, O = lin.T, lin.I, lin.O
+            Q = B.QuantizedTensor
+            layer = {
+                "lin": lin, **tens,
+                "fprop": (Q(T, I, device), Q(O, I, device)),
+                "dgrad": (Q(T, O, device), Q(I, O, device)),
+                "wgrad": (Q(O, T, device), Q(I, T, device)),
+                "out": {"fprop": torch.empty((T, O), dtype=torch.bfloat16, device=device),
+                        "dgrad": torch.empty((T, I), dtype=torch.bfloat16, device=device),
+                        "wgrad": torch.empty((O, I), dtype=torch.float32, device=device)},
+            }
+            self.layers.append(layer)
+        self.workspace = torch.empty((B.workspace_bytes(1 << 14, 1 << 14),), dtype=torch.uint8,
+                                     device=device)
+        self.dev_status = torch.zeros(1, dtype=torch.int32, device=device)
+        self.flops_per_gemm = [2 * L["lin"].T * L["lin"].I * L["lin"].O for L in self.layers]
+
+    @property
+    def gemm_flops(self):
+        return sum(3 * f for f in self.flops_per_gemm)
+
+    def quant_bytes(self):
+        """Algorithmic quantizer bytes of one step: per operand, the amax read (2 B/elem),
+        the quantize read (2 B/elem) and the codes + scales write (0.5 + 1/16 B/elem)."""
+        total = 0
+        for L in self.layers:
+            lin = L["lin"]
+            for n in (lin.T * lin.I, lin.O * lin.I, lin.T * lin.O, lin.O * lin.I,
+                      lin.T * lin.O, lin.T * lin.I):
+                total += n * (2 + 2 + 0.5 + 1 / 16)
+        return total
+
+    def n_quant_launches(self):
+        return 2 * 2 * 3 * len(self.layers)   # (amax + quantize) x 2 operands x 3 GEMMs
+
+    def n_gemm_launches(self):
+        return 3 * len(self.layers)
+
+    def run(self, events=None):
+        """Queue one step on the current stream.  With `events`, record CUDA events around
+        every GEMM (events['gemm']) and every operand quantization (events['quant'])."""
+        B = self.B
+        ws, st = self.workspace, self.dev_status
+
+        def timed(kind, fn):
+            if events is None:
+                fn()
+                return
+            e0 = self.torch.cuda.Event(enable_timing=True)
+            e1 = self.torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            events[kind].append((e0, e1))
+
+        for L in self.layers:
+            X, W, dY, out = L["X"], L["W"], L["dY"], L["out"]
+            a, b = L["fprop"]
+            timed("quant", lambda: B.quantize(W, B.ROWWISE | B.BLOCK2D, out_row=b, workspace=ws,
+                                              dev_status=st))
+            timed("quant", lambda: B.quantize(X, B.ROWWISE, out_row=a, workspace=ws,
+                                              dev_status=st))
+            timed("gemm", lambda: B.gemm(a, b, out=out["fprop"], dev_status=st))
+            a, b = L["dgrad"]
+            timed("quant", lambda: B.quantize(W, B.COLWISE | B.BLOCK2D, out_col=b, workspace=ws,
+                                              dev_status=st))
+            timed("quant", lambda: B.quantize(dY, B.ROWWISE | B.SR, seed=self.seed, offset=0,
+                                              out_row=a, workspace=ws, dev_status=st))
+            timed("gemm", lambda: B.gemm(a, b, out=out["dgrad"], dev_status=st))
+            a, b = L["wgrad"]
+            timed("quant", lambda: B.rht_quantize(dY, self.mask, B.SR, seed=self.seed, offset=1,
+                                                  out_col=a, workspace=ws, dev_status=st))
+            timed("quant", lambda: B.rht_quantize(X, self.mask, 0, out_col=b, workspace=ws,
+                                                  dev_status=st))
+            timed("gemm", lambda: B.gemm(a, b, out=out["wgrad"], dev_status=st))
+
+    def upload(self):
+        """Host -> device copies of this step's inputs (from pinned memory)."""
+        i = 0
+        for L in self.layers:
+            for name in ("X", "W", "dY"):
+                L[name].copy_(self.host[i], non_blocking=True)
+                i += 1
+
+    def h2d_bytes(self):
+        return sum(h.numel() * h.element_size() for h in self.host)
+
+    def download(self, outs_host):
+        i = 0
+        for L in self.layers:
+            for op in OPS:
+                outs_host[i].copy_(L["out"][op], non_blocking=True)
+                i += 1
+
+    def output_host_buffers(self):
+        bufs = []
+        for L in self.layers:
+            for op in OPS:
+                o = L["out"][op]
+                bufs.append(self.torch.empty(o.shape, dtype=o.dtype).pin_memory())
+        return bufs
+
+
+# ---- CPU oracle leg ----------------------------------------------------------------------
+
+def oracle_sample(workload, tokens=128, max_out=512, max_in=4096):
+    """Time the CPU oracle on a bounded sample of the workload: for every linear, the first
+    `tokens` tokens, the first min(O, max_out) out-features and min(I, max_in) in-features;
+    the three GEMMs' operand quantizations and FP64 reference products.  Returns
+    (seconds, GEMM flops of the sample, threads used)."""
+    import oracle
+    flops = 0
+    t0 = time.perf_counter()
+    for li, lin in enumerate(workload.linears):
+        X, W, dY = synth.linear_inputs(lin, workload.seed, layer_index=li)
+        Ts, Is, Os = tokens, min(lin.I, max_in), min(lin.O, max_out)
+        Xs = np.ascontiguousarray(X[:Ts, :Is])
+        Ws = np.ascontiguousarray(W[:Os, :Is])
+        dYs = np.ascontiguousarray(dY[:Ts, :Os])
+        mask = oracle.sign_mask_from_seed(workload.seed)
+        for qa, qb in (oracle.fprop_operands(Xs, Ws),
+                       oracle.dgrad_operands(dYs, Ws, workload.seed, 0),
+                       oracle.wgrad_operands(dYs, Xs, mask, workload.seed, 0)):
+            oracle.gemm_ref(qa, qb)
+            flops += 2 * qa.rows * qb.rows * qa.cols
+    secs = time.perf_counter() - t0
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        threads = 1
+    return secs, flops, threads
+
+
+def cpu_baseline(workload):
+    secs, flops, threads = oracle_sample(workload)
+    return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": "per linear: first 128 tokens, first min(O,512) out- and min(I,4096) "
+                      "in-features; fprop/dgrad/wgrad operand quantization (C oracle) + FP64 "
+                      "reference GEMM (numpy matmul of dequantized operands)",
+            "seconds": secs}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    wl = synth.mlp_12b()
+    for _ in range(args.warmup):
+        oracle_sample(wl, tokens=64, max_out=256, max_in=2048)
+    times, flops, threads = [], 0, 1
+    for _ in range(args.steps):
+        secs, flops, threads = oracle_sample(wl, tokens=64, max_out=256, max_in=2048)
+        times.append(secs)
+    total = sum(times)
+    value = flops * len(times) / total / 1e12
+    sample = ("per linear: first 64 tokens, first min(O,256) out- and min(I,2048) in-features; "
+              "operand quantization (C oracle) + FP64 reference GEMMs")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": wl.name, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- GPU leg -----------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    device = torch.device("cuda", local if world > 1 else torch.cuda.current_device())
+    torch.cuda.set_device(device)
+    peaks = _peaks()
+    wl = synth.mlp_12b()
+    step = Step(wl, device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    st = int(step.dev_status.item())
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    events = {"gemm": [], "quant": []}
+    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(args.steps):
+            step.run(events)
+        t1.record()
+        torch.cuda.synchronize()
+        barrier()
+    ms_local = t0.elapsed_time(t1) / args.steps
+    ms = max_over_ranks(ms_local, device)
+    value = whole_job_rate(step.gemm_flops / 1e12, world, ms / 1e3)
+
+    gemm_ms = [a.elapsed_time(b) for a, b in events["gemm"]]
+    quant_ms = [a.elapsed_time(b) for a, b in events["quant"]]
+    gemm_avg_ms = sum(gemm_ms) / len(gemm_ms)
+    flops_per_launch = step.flops_per_gemm[0]  # every GEMM of this workload: 2*8192*5120*20480
+    achieved = flops_per_launch / (gemm_avg_ms / 1e3) / 1e12
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    quant_gbs = step.quant_bytes() * args.steps / (sum(quant_ms) / 1e3) / 1e9
+
+    # end-to-end: inputs from pinned host memory, outputs back to pinned host memory
+    e2e = None
+    if not args.no_e2e:
+        outs = step.output_host_buffers()
+        e2e_steps = max(1, min(args.steps, 5))
+        barrier()
+        torch.cuda.synchronize()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        s0.record()
+        for _ in range(e2e_steps):
+            step.upload()
+            step.run()
+            step.download(outs)
+        s1.record()
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(s0.elapsed_time(s1) / e2e_steps, device)
+        d2h = sum(o.numel() * o.element_size() for o in outs)
+        e2e = {"value": whole_job_rate(step.gemm_flops / 1e12, world, e2e_ms / 1e3),
+               "unit": "TFLOP/s", "h2d_bytes_per_step": step.h2d_bytes(),
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl)
+
+    st = int(step.dev_status.item())
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
+            "data": "synthetic: seeded N(0,1) activations with 1% x50 outliers, N(0,0.02) "
+                    "random-init weights, N(0,1e-3) gradients with 0.5% x100 spikes",
+            "config": {"workload": wl.name, "tokens": 8192, "d_model": 5120, "d_ff": 20480,
+                       "gemms_per_step": 6, "gemm_tflop_per_step": step.gemm_flops / 1e12,
+                       "outputs": "Y and dX bf16, dW fp32",
+                       "recipe": "W 16x16 RTN, X 1x16 RTN, dY 1x16 SR, wgrad RHT16 (+SR on dY)",
+                       "l2": "inputs larger than L2: 1.26 GB of bf16 inputs read per step",
+                       "parallelism": "replicas" if world > 1 else "single GPU"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": None,
+                         "kernel": "gemm_nvf4_kernel",
+                         "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} "
+                                        f"TFLOP/s x {FP4_OVER_BF16:g} (nominal FP4:BF16)",
+                         "avg_launch_ms": gemm_avg_ms},
+            "quantize": {"gbps": quant_gbs, "peak_gbs": peaks["hbm_gbs"],
+                         "frac": quant_gbs / peaks["hbm_gbs"],
+                         "bytes_per_step": step.quant_bytes(),
+                         "ms_per_step": sum(quant_ms) / args.steps},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": (step.n_gemm_launches() + step.n_quant_launches()) * args.steps,
+            "clocks": clocks.summary(),
+            "dev_status": st,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0 if st == 0 else 1
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

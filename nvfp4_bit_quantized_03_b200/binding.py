@@ -1,0 +1,250 @@
+"""ctypes binding of libnvfp4.so (include/nvfp4.h).
+
+Argument marshalling only: PyTorch owns the device memory and the streams; every step of the
+quantizers and GEMMs runs in the library's CUDA kernels.  There is no fallback: if the
+library is missing or a call fails, an exception is raised.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "nvfp4.h")
+
+# status codes and flags (include/nvfp4.h)
+OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_DEVICE, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_ARG = range(9)
+DEVSTAT_NONFINITE, DEVSTAT_TIMEOUT = 1, 2
+ROWWISE, COLWISE, BLOCK2D, SR, AMAX_GIVEN = 1, 2, 4, 8, 16
+OUT_F32, OUT_BF16 = 0, 1
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {lib().nvfp4_status_string(status).decode()} (status {status})")
+
+
+class Operand(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("amax", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libnvfp4.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libnvfp4.so not found at {LIB_PATH}; build it with "
+                              "`python -m nvfp4_bit_quantized_03_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(LIB_PATH)
+        i64, u64, u16, vp, i32 = (ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint16,
+                                  ctypes.c_void_p, ctypes.c_int)
+        op = ctypes.POINTER(Operand)
+        sz = ctypes.c_size_t
+        L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
+        L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
+        L.nvfp4_codes_bytes.argtypes, L.nvfp4_codes_bytes.restype = [i64, i64], sz
+        L.nvfp4_scales_bytes.argtypes, L.nvfp4_scales_bytes.restype = [i64, i64], sz
+        L.nvfp4_workspace_bytes.argtypes = [i64, i64, ctypes.c_uint]
+        L.nvfp4_workspace_bytes.restype = sz
+        L.nvfp4_linear_workspace_bytes.argtypes = [i64, i64, i64]
+        L.nvfp4_linear_workspace_bytes.restype = sz
+        L.nvfp4_sign_mask_from_seed.argtypes, L.nvfp4_sign_mask_from_seed.restype = [u64], u16
+        L.nvfp4_scales_unswizzle.argtypes = [vp, i64, i64, vp]
+        L.nvfp4_scales_unswizzle.restype = i32
+        L.nvfp4_quantize.argtypes = [vp, i64, i64, i64, ctypes.c_uint, u64, u64, op, op, vp, vp, vp]
+        L.nvfp4_quantize.restype = i32
+        L.nvfp4_rht_quantize.argtypes = [vp, i64, i64, i64, u16, ctypes.c_uint, u64, u64, op, vp,
+                                         vp, vp]
+        L.nvfp4_rht_quantize.restype = i32
+        L.nvfp4_gemm.argtypes = [op, op, vp, i32, i64, vp, vp]
+        L.nvfp4_gemm.restype = i32
+        L.nvfp4_linear_fprop.argtypes = [vp, vp, i64, i64, i64, vp, i32, vp, vp, vp]
+        L.nvfp4_linear_fprop.restype = i32
+        L.nvfp4_linear_dgrad.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, i32, vp, vp, vp]
+        L.nvfp4_linear_dgrad.restype = i32
+        L.nvfp4_linear_wgrad.argtypes = [vp, vp, i64, i64, i64, u16, u64, u64, vp, i32, vp, vp, vp]
+        L.nvfp4_linear_wgrad.restype = i32
+        _lib = L
+    return _lib
+
+
+def declared_functions():
+    """Names of the functions include/nvfp4.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", text)))
+
+
+def _check(status, what):
+    if status != OK:
+        raise NVFP4Error(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+# ---- sizes and host helpers -------------------------------------------------------------
+
+def codes_bytes(rows, cols):
+    return lib().nvfp4_codes_bytes(rows, cols)
+
+
+def scales_bytes(rows, cols):
+    return lib().nvfp4_scales_bytes(rows, cols)
+
+
+def workspace_bytes(rows, cols, flags=0):
+    return lib().nvfp4_workspace_bytes(rows, cols, flags)
+
+
+def linear_workspace_bytes(T, I, O):
+    return lib().nvfp4_linear_workspace_bytes(T, I, O)
+
+
+def sign_mask_from_seed(seed):
+    return lib().nvfp4_sign_mask_from_seed(seed)
+
+
+def scales_unswizzle(swizzled, rows, cols):
+    """Host (numpy uint8) MMA-layout scales -> row-major [rows x cols/16]."""
+    import numpy as np
+    src = np.ascontiguousarray(swizzled, dtype=np.uint8)
+    out = np.zeros((rows, cols // 16), dtype=np.uint8)
+    _check(lib().nvfp4_scales_unswizzle(src.ctypes.data_as(ctypes.c_void_p), rows, cols,
+                                        out.ctypes.data_as(ctypes.c_void_p)), "scales_unswizzle")
+    return out
+
+
+# ---- device buffers ---------------------------------------------------------------------
+
+class QuantizedTensor:
+    """A quantized operand whose buffers torch allocated: codes [rows x cols/2] uint8,
+    scales (MMA layout) uint8, amax float32[1]."""
+
+    def __init__(self, rows, cols, device="cuda"):
+        self.rows, self.cols = rows, cols
+        self.codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
+        self.scales = torch.empty((scales_bytes(rows, cols),), dtype=torch.uint8, device=device)
+        self.amax = torch.zeros((1,), dtype=torch.float32, device=device)
+
+    def operand(self):
+        return Operand(self.codes.data_ptr(), self.scales.data_ptr(), self.amax.data_ptr(),
+                       self.rows, self.cols)
+
+
+def _workspace(nbytes, device):
+    if nbytes == 0:
+        return None
+    return torch.empty((nbytes,), dtype=torch.uint8, device=device)
+
+
+def quantize(x, flags, seed=0, offset=0, out_row=None, out_col=None, workspace=None,
+             dev_status=None, stream=None):
+    """nvfp4_quantize on a 2D bf16 CUDA tensor (row stride x.stride(0))."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if flags & ROWWISE and out_row is None:
+        out_row = QuantizedTensor(rows, cols, x.device)
+    if flags & COLWISE and out_col is None:
+        out_col = QuantizedTensor(cols, rows, x.device)
+    if workspace is None:
+        workspace = _workspace(workspace_bytes(rows, cols, flags), x.device)
+    op_r = out_row.operand() if out_row is not None else None
+    op_c = out_col.operand() if out_col is not None else None
+    st = lib().nvfp4_quantize(_ptr(x), rows, cols, x.stride(0), flags, seed, offset,
+                              ctypes.byref(op_r) if op_r is not None else None,
+                              ctypes.byref(op_c) if op_c is not None else None,
+                              _ptr(workspace), _ptr(dev_status), _stream(stream))
+    _check(st, "nvfp4_quantize")
+    return out_row, out_col
+
+
+def rht_quantize(x, sign_mask, flags=0, seed=0, offset=0, out_col=None, workspace=None,
+                 dev_status=None, stream=None):
+    """nvfp4_rht_quantize: x^T random-Hadamard-transformed and quantized along x's rows."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out_col is None:
+        out_col = QuantizedTensor(cols, rows, x.device)
+    if workspace is None:
+        workspace = _workspace(workspace_bytes(rows, cols, flags), x.device)
+    op_c = out_col.operand()
+    st = lib().nvfp4_rht_quantize(_ptr(x), rows, cols, x.stride(0), sign_mask, flags, seed,
+                                  offset, ctypes.byref(op_c), _ptr(workspace), _ptr(dev_status),
+                                  _stream(stream))
+    _check(st, "nvfp4_rht_quantize")
+    return out_col
+
+
+def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None):
+    """nvfp4_gemm: D = A . B^T (A, B QuantizedTensor)."""
+    d_dtype = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
+    if out is None:
+        out = torch.empty((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
+    oa, ob = A.operand(), B.operand()
+    st = lib().nvfp4_gemm(ctypes.byref(oa), ctypes.byref(ob), _ptr(out), d_dtype, out.stride(0),
+                          _ptr(dev_status), _stream(stream))
+    _check(st, "nvfp4_gemm")
+    return out
+
+
+def _dtype_code(dtype):
+    return OUT_F32 if dtype == torch.float32 else OUT_BF16
+
+
+def linear_fprop(X, W, out=None, out_dtype=torch.float32, workspace=None, dev_status=None,
+                 stream=None):
+    T, I = X.shape
+    O = W.shape[0]
+    if out is None:
+        out = torch.empty((T, O), dtype=out_dtype, device=X.device)
+    if workspace is None:
+        workspace = _workspace(linear_workspace_bytes(T, I, O), X.device)
+    st = lib().nvfp4_linear_fprop(_ptr(X), _ptr(W), T, I, O, _ptr(out), _dtype_code(out.dtype),
+                                  _ptr(workspace), _ptr(dev_status), _stream(stream))
+    _check(st, "nvfp4_linear_fprop")
+    return out
+
+
+def linear_dgrad(dY, W, seed, offset, out=None, out_dtype=torch.float32, workspace=None,
+                 dev_status=None, stream=None):
+    T, O = dY.shape
+    I = W.shape[1]
+    if out is None:
+        out = torch.empty((T, I), dtype=out_dtype, device=dY.device)
+    if workspace is None:
+        workspace = _workspace(linear_workspace_bytes(T, I, O), dY.device)
+    st = lib().nvfp4_linear_dgrad(_ptr(dY), _ptr(W), T, I, O, seed, offset, _ptr(out),
+                                  _dtype_code(out.dtype), _ptr(workspace), _ptr(dev_status),
+                                  _stream(stream))
+    _check(st, "nvfp4_linear_dgrad")
+    return out
+
+
+def linear_wgrad(dY, X, sign_mask, seed, offset, out=None, out_dtype=torch.float32,
+                 workspace=None, dev_status=None, stream=None):
+    T, O = dY.shape
+    I = X.shape[1]
+    if out is None:
+        out = torch.empty((O, I), dtype=out_dtype, device=dY.device)
+    if workspace is None:
+        workspace = _workspace(linear_workspace_bytes(T, I, O), dY.device)
+    st = lib().nvfp4_linear_wgrad(_ptr(dY), _ptr(X), T, I, O, sign_mask, seed, offset, _ptr(out),
+                                  _dtype_code(out.dtype), _ptr(workspace), _ptr(dev_status),
+                                  _stream(stream))
+    _check(st, "nvfp4_linear_wgrad")
+    return out

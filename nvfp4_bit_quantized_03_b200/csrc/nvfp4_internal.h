@@ -1,0 +1,62 @@
+// Internal interfaces between the C ABI (api.cu) and the kernels (quantize.cu, gemm.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+namespace nvfp4 {
+
+// Upper bound on the CTAs of the amax pass, i.e. on the partial maxima in the workspace.
+constexpr int kMaxPartials = 2048;
+
+// Where a quantize kernel gets the tensor amax from: the partial maxima written by the
+// amax pass (FP32 bit patterns), or a caller-given FP32 value.
+struct QuantSource {
+    const uint32_t* partials;
+    int n_partials;
+    const float* amax_given;  // non-null: use *amax_given, ignore the partials
+};
+
+struct TileArgs {
+    const uint16_t* x;
+    int64_t rows, cols, ld;
+    QuantSource src;
+    uint8_t* row_codes;
+    uint8_t* row_scales;
+    float* row_amax;
+    uint8_t* col_codes;
+    uint8_t* col_scales;
+    float* col_amax;
+    uint32_t sign_mask;
+    uint64_t seed, offset;
+    int* dev_status;
+};
+
+int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count);
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool rht,
+                        uint32_t sign_mask, uint32_t* partials, int grid, cudaStream_t s);
+cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                 const QuantSource& src, float* amax_out0, float* amax_out1,
+                                 uint8_t* codes, uint8_t* scales, bool sr, uint64_t seed,
+                                 uint64_t offset, int* dev_status, int sm_count, cudaStream_t s);
+cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2d, bool rht,
+                              bool sr, int sm_count, cudaStream_t s);
+
+struct GemmArgs {
+    const uint8_t* a_codes;
+    const uint8_t* a_scales;
+    const float* a_amax;
+    const uint8_t* b_codes;
+    const uint8_t* b_scales;
+    const float* b_amax;
+    int64_t M, N, K;
+    void* D;
+    int64_t ldd;
+    int out_bf16;
+    int* dev_status;
+};
+
+cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s);
+
+}  // namespace nvfp4

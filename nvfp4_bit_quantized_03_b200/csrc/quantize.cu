@@ -1,0 +1,455 @@
+// NVFP4 quantizer kernels for sm_100a.
+//
+// Method: "Pretraining Large Language Models with NVFP4" (gist.science summary), Resumen
+// tecnico section 2, "Formato NVFP4" (E2M1 elements in 16-element blocks, E4M3 block scale,
+// FP32 tensor scale), "Transformadas de Hadamard Aleatorias (RHT)" (16x16 Hadamard with a
+// fixed random sign vector on the weight-gradient inputs) and "Escalado Bidimensional (2D)
+// y Redondeo Estocastico" (16x16 weight blocks; stochastic rounding of gradients).
+//
+// Two passes over the bf16 input, both HBM-bound streams:
+//   1. amax_kernel / amax_rht_kernel: per-CTA partial maxima of |x| (or |RHT(x)|) into the
+//      workspace.  The plain pass compares bf16 magnitude bit patterns (exact).
+//   2. quant_rowwise_kernel (1x16 blocks along the row, coalesced 16-byte loads, block max
+//      by one warp shuffle, one Philox call per 8 elements for SR) or quant_tile_kernel
+//      (64 x 128 tiles staged in shared memory for the column-wise / transposed outputs,
+//      16x16 weight tiles and the fused RHT).  Each CTA first folds the partial maxima into
+//      the tensor amax.  The second pass walks the tensor in the reverse order of the
+//      first, so the tail the first pass left in L2 is re-read from L2.
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "nvfp4_device.cuh"
+#include "nvfp4_internal.h"
+
+namespace nvfp4 {
+
+// ------------------------------------------------------------------------------------------
+// Pass 1: amax
+// ------------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                   int64_t cols, int64_t ld,
+                                                   uint32_t* __restrict__ partials)
+{
+    const int64_t cpr = cols >> 3;  // 16-byte chunks per row
+    const int64_t total = rows * cpr;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    uint32_t m = 0;
+    if (ld == cols) {
+        const uint4* p = reinterpret_cast<const uint4*>(x);
+        for (; i + 3 * stride < total; i += 4 * stride) {
+            const uint4 a = __ldg(p + i), b = __ldg(p + i + stride);
+            const uint4 c = __ldg(p + i + 2 * stride), d = __ldg(p + i + 3 * stride);
+            m = max(m, max(max(absmax_bits8(a), absmax_bits8(b)),
+                           max(absmax_bits8(c), absmax_bits8(d))));
+        }
+        for (; i < total; i += stride) m = max(m, absmax_bits8(__ldg(p + i)));
+    } else {
+        for (; i < total; i += stride) {
+            const int64_t r = i / cpr, c = i - r * cpr;
+            m = max(m, absmax_bits8(__ldg(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+        }
+    }
+    block_max_store(m, partials + blockIdx.x);
+}
+
+// amax of the random Hadamard transform along the rows: each work item is 16 rows x 8
+// columns (16 coalesced 16-byte loads), i.e. eight 16-element transforms.
+__global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x,
+                                                       int64_t rows, int64_t cols, int64_t ld,
+                                                       uint32_t sign_mask,
+                                                       uint32_t* __restrict__ partials)
+{
+    const int64_t cpr = cols >> 3;
+    const int64_t total = (rows >> 4) * cpr;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    uint32_t m = 0;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+         i += stride) {
+        const int64_t g = i / cpr, c = i - g * cpr;
+        const uint16_t* base = x + (g << 4) * ld + (c << 3);
+        uint4 v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = __ldg(reinterpret_cast<const uint4*>(base + k * ld));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            float y[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const uint32_t w = j < 2 ? v[k].x : j < 4 ? v[k].y : j < 6 ? v[k].z : v[k].w;
+                y[k] = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+            }
+            rht16(y, sign_mask);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) m = max(m, __float_as_uint(fabsf(y[k])));
+        }
+    }
+    block_max_store(m, partials + blockIdx.x);
+}
+
+// ------------------------------------------------------------------------------------------
+// Shared prologue of the quantize kernels: the tensor amax and its encode scale.
+// ------------------------------------------------------------------------------------------
+struct TensorScale {
+    float s_enc;
+    bool nonfinite;
+};
+
+__device__ __forceinline__ TensorScale fold_amax(const QuantSource& src, float* amax_out0,
+                                                 float* amax_out1, int* dev_status)
+{
+    uint32_t bits;
+    if (src.amax_given) {
+        const float a = *src.amax_given;
+        const bool bad = !(a >= 0.0f) || a == INFINITY;
+        bits = bad ? kF32InfBits : __float_as_uint(a + 0.0f);  // +0.0f folds -0 into +0
+    } else {
+        bits = reduce_partials(src.partials, src.n_partials);
+    }
+    TensorScale ts;
+    ts.nonfinite = bits >= kF32InfBits;
+    ts.s_enc = ts.nonfinite ? 1.0f : tensor_scale(__uint_as_float(bits));
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        const float amax = ts.nonfinite ? INFINITY : __uint_as_float(bits);
+        if (!src.amax_given || ts.nonfinite) {
+            if (amax_out0) *amax_out0 = amax;
+            if (amax_out1) *amax_out1 = amax;
+        } else if (amax_out1 && amax_out1 != src.amax_given) {
+            *amax_out1 = amax;
+        }
+        if (ts.nonfinite && dev_status) atomicOr(dev_status, static_cast<int>(kDevNonfinite));
+    }
+    return ts;
+}
+
+// Zero the scale words of the padding rows [rows, rows_pad) of a scale buffer.
+__device__ __forceinline__ void zero_scale_padding(uint8_t* scales, int64_t rows, int64_t cols,
+                                                   int64_t first_item, int64_t item_stride)
+{
+    const int64_t gpr = cols >> 6;  // 4-block groups per row
+    const int64_t rows_pad = (rows + 127) & ~static_cast<int64_t>(127);
+    const int64_t n = (rows_pad - rows) * gpr;
+    for (int64_t i = first_item; i < n; i += item_stride) {
+        const int64_t r = rows + i / gpr, g = i % gpr;
+        *reinterpret_cast<uint32_t*>(scales + sf_offset(r, g << 2, gpr)) = 0u;
+    }
+}
+
+// ------------------------------------------------------------------------------------------
+// Pass 2a: row-wise 1x16 quantization (x quantized along its columns).
+// Lane l of a warp owns 16-byte chunk (base + l): 8 elements; the two lanes of a 16-element
+// block exchange their maxima with one shuffle; lane 8k gathers the 4 scales of its
+// 64-element group into one 32-bit word.  With SR the Philox counter of the chunk is its
+// flat index (element index / 8).
+// ------------------------------------------------------------------------------------------
+template <bool SR>
+__global__ void __launch_bounds__(256) quant_rowwise_kernel(
+    const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, QuantSource src,
+    float* amax_out0, float* amax_out1, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, uint64_t seed, uint64_t offset, int* dev_status)
+{
+    const TensorScale ts = fold_amax(src, amax_out0, amax_out1, dev_status);
+    const Philox philox(seed);
+    const int lane = threadIdx.x & 31;
+    const int64_t cpr = cols >> 3;
+    const int64_t gpr = cols >> 6;
+    const int64_t total = rows * cpr;                   // chunks (multiple of 8)
+    const int64_t nwork = (total + 31) >> 5;            // warp-sized pieces
+    const int64_t wstride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    const int64_t wfirst = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+
+    for (int64_t w = wfirst; w < nwork; w += wstride) {
+        const int64_t f = ((nwork - 1 - w) << 5) + lane;  // reverse order (L2 reuse)
+        const bool valid = f < total;
+        int64_t r = 0, c8 = 0;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (valid) {
+            r = f / cpr;
+            c8 = f - r * cpr;
+            v = __ldg(reinterpret_cast<const uint4*>(x + r * ld) + c8);
+        }
+        float e[8];
+        unpack8(v, e);
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(e[j]));
+        const float b = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        const BlockScale bs = block_scale(b, ts.s_enc);
+        uint32_t packed = 0;
+        if (SR) {
+            const uint4 rnd = philox.group(static_cast<uint64_t>(f), offset);
+#pragma unroll
+            for (int j = 0; j < 8; j += 2) {
+                const float q0 = e2m1_sr_value(__fmul_rn(e[j], bs.r), lane16(rnd, j));
+                const float q1 = e2m1_sr_value(__fmul_rn(e[j + 1], bs.r), lane16(rnd, j + 1));
+                packed |= e2m1x2_rn(q0, q1) << (4 * j);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; j += 2)
+                packed |= e2m1x2_rn(__fmul_rn(e[j], bs.r), __fmul_rn(e[j + 1], bs.r)) << (4 * j);
+        }
+        const uint32_t sf = ts.nonfinite ? 0u : bs.sf;
+        if (ts.nonfinite) packed = 0;
+        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sf, 2);
+        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sf, 4);
+        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sf, 6);
+        if (valid) {
+            reinterpret_cast<uint32_t*>(codes)[f] = packed;
+            if ((lane & 7) == 0)
+                *reinterpret_cast<uint32_t*>(scales + sf_offset(r, c8 >> 1, gpr)) =
+                    sf | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        }
+    }
+    zero_scale_padding(scales, rows, cols,
+                       static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
+                       static_cast<int64_t>(gridDim.x) * blockDim.x);
+}
+
+// ------------------------------------------------------------------------------------------
+// Pass 2b: tile quantizer.  A CTA stages a 64-row x 128-column tile in shared memory (rows
+// padded to 136 elements so both the row and the column walks are free of bank conflicts)
+// and produces
+//   ROW: the row-wise output (blocks along the columns), thread t -> row t % 64, blocks
+//        4 (t / 64) .. +3: 32 contiguous code bytes and one scale word;
+//   COL: the column-wise output (x^T, blocks along the rows, optionally RHT'd), thread t ->
+//        column t, the tile's 4 row blocks: 32 contiguous code bytes and one scale word.
+// BLOCK2D: the scale of every 16x16 sub-tile comes from its maximum, shared by both outputs,
+// whose codes are then the same nibbles transposed.
+// ------------------------------------------------------------------------------------------
+constexpr int kTileRows = 64, kTileCols = 128, kTilePitch = 136;
+
+template <bool SR>
+__device__ __forceinline__ void encode16(const float* y, const BlockScale& bs, const Philox& ph,
+                                         uint64_t e0, uint64_t offset, uint32_t& w0,
+                                         uint32_t& w1)
+{
+    uint32_t p[2] = {0u, 0u};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint4 rnd = make_uint4(0, 0, 0, 0);
+        if (SR) rnd = ph.group((e0 >> 3) + h, offset);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            float a = __fmul_rn(y[8 * h + j], bs.r), b = __fmul_rn(y[8 * h + j + 1], bs.r);
+            if (SR) {
+                a = e2m1_sr_value(a, lane16(rnd, j));
+                b = e2m1_sr_value(b, lane16(rnd, j + 1));
+            }
+            p[h] |= e2m1x2_rn(a, b) << (4 * j);
+        }
+    }
+    w0 = p[0];
+    w1 = p[1];
+}
+
+template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR>
+__global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
+{
+    __shared__ __align__(16) uint16_t tile[kTileRows * kTilePitch];
+    __shared__ float bmax[kTileRows][8];
+    __shared__ float tmax[4][8];
+
+    const TensorScale ts = fold_amax(a.src, ROW ? a.row_amax : a.col_amax,
+                                     ROW ? a.col_amax : nullptr, a.dev_status);
+    const Philox philox(a.seed);
+    const int t = threadIdx.x;
+    const int64_t tiles_c = (a.cols + kTileCols - 1) / kTileCols;
+    const int64_t tiles_r = (a.rows + kTileRows - 1) / kTileRows;
+    const int64_t ntiles = tiles_c * tiles_r;
+
+    for (int64_t id = blockIdx.x; id < ntiles; id += gridDim.x) {
+        const int64_t tid = ntiles - 1 - id;  // reverse order (L2 reuse)
+        const int64_t r0 = (tid / tiles_c) * kTileRows, c0 = (tid % tiles_c) * kTileCols;
+        const int nr = static_cast<int>(a.rows - r0 < kTileRows ? a.rows - r0 : kTileRows);
+        const int nc = static_cast<int>(a.cols - c0 < kTileCols ? a.cols - c0 : kTileCols);
+
+        __syncthreads();  // the previous tile's readers are done with `tile`
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int ch = t + 128 * k, row = ch >> 4, cc = ch & 15;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (row < nr && cc * 8 < nc)
+                v = __ldg(reinterpret_cast<const uint4*>(a.x + (r0 + row) * a.ld + c0) + cc);
+            *reinterpret_cast<uint4*>(tile + row * kTilePitch + cc * 8) = v;
+        }
+        __syncthreads();
+
+        // Row walk: thread t -> row t % 64, blocks 4 (t / 64) .. +3.
+        const int rrow = t & 63, rblk = (t >> 6) * 4;
+        float rv[4][16];
+        float rb[4];
+        if (ROW || BLOCK2D) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint16_t* src = tile + rrow * kTilePitch + (rblk + q) * 16;
+                const uint4 lo = *reinterpret_cast<const uint4*>(src);
+                const uint4 hi = *reinterpret_cast<const uint4*>(src + 8);
+                unpack8(lo, rv[q]);
+                unpack8(hi, rv[q] + 8);
+                float m = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(rv[q][j]));
+                rb[q] = m;
+                if (BLOCK2D) bmax[rrow][rblk + q] = m;
+            }
+        }
+        if (BLOCK2D) {
+            __syncthreads();
+            if (t < 32) {
+                const int tr = t >> 3, tc = t & 7;
+                float m = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) m = fmaxf(m, bmax[tr * 16 + i][tc]);
+                tmax[tr][tc] = m;
+            }
+            __syncthreads();
+        }
+
+        if (ROW && rrow < nr && rblk * 16 < nc) {
+            const int64_t r = r0 + rrow;
+            uint32_t words[8];
+            uint32_t sfw = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float b = BLOCK2D ? tmax[rrow >> 4][rblk + q] : rb[q];
+                const BlockScale bs = block_scale(b, ts.s_enc);
+                const uint64_t e0 = static_cast<uint64_t>(r) * a.cols + c0 + (rblk + q) * 16;
+                encode16<SR>(rv[q], bs, philox, e0, a.offset, words[2 * q], words[2 * q + 1]);
+                sfw |= bs.sf << (8 * q);
+            }
+            if (ts.nonfinite) {
+                sfw = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) words[q] = 0;
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.row_codes + (r * a.cols + c0 + rblk * 16) / 2);
+            dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+            dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+            *reinterpret_cast<uint32_t*>(a.row_scales +
+                                         sf_offset(r, (c0 >> 4) + rblk, a.cols >> 6)) = sfw;
+        }
+
+        if (COL && t < nc) {
+            const int64_t orow = c0 + t;  // output row = input column
+            uint32_t words[8];
+            uint32_t sfw = 0;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float y[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    y[i] = __uint_as_float(static_cast<uint32_t>(
+                               tile[(q * 16 + i) * kTilePitch + t]) << 16);
+                if (RHT) rht16(y, a.sign_mask);
+                float b;
+                if (BLOCK2D) {
+                    b = tmax[q][t >> 4];
+                } else {
+                    b = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(y[i]));
+                }
+                const BlockScale bs = block_scale(b, ts.s_enc);
+                const uint64_t e0 = static_cast<uint64_t>(orow) * a.rows + r0 + q * 16;
+                encode16<SR>(y, bs, philox, e0, a.offset, words[2 * q], words[2 * q + 1]);
+                sfw |= bs.sf << (8 * q);
+            }
+            if (ts.nonfinite) {
+                sfw = 0;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) words[q] = 0;
+            }
+            uint4* dst = reinterpret_cast<uint4*>(a.col_codes + (orow * a.rows + r0) / 2);
+            dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+            dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+            *reinterpret_cast<uint32_t*>(a.col_scales + sf_offset(orow, r0 >> 4, a.rows >> 6)) =
+                sfw;
+        }
+    }
+    const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    if (ROW) zero_scale_padding(a.row_scales, a.rows, a.cols, first, step);
+    if (COL) zero_scale_padding(a.col_scales, a.cols, a.rows, first, step);
+}
+
+// ------------------------------------------------------------------------------------------
+// Launchers
+// ------------------------------------------------------------------------------------------
+
+int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count)
+{
+    const int64_t items = rht ? (rows / 16) * (cols / 8) : rows * (cols / 8);
+    const int64_t per_cta = rht ? 256 : 256 * 4;
+    int64_t g = (items + per_cta - 1) / per_cta;
+    const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+    if (g > cap) g = cap;
+    if (g > kMaxPartials) g = kMaxPartials;
+    if (g < 1) g = 1;
+    return static_cast<int>(g);
+}
+
+cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool rht,
+                        uint32_t sign_mask, uint32_t* partials, int grid, cudaStream_t s)
+{
+    if (rht)
+        amax_rht_kernel<<<grid, 256, 0, s>>>(x, rows, cols, ld, sign_mask, partials);
+    else
+        amax_kernel<<<grid, 256, 0, s>>>(x, rows, cols, ld, partials);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                                 const QuantSource& src, float* amax_out0, float* amax_out1,
+                                 uint8_t* codes, uint8_t* scales, bool sr, uint64_t seed,
+                                 uint64_t offset, int* dev_status, int sm_count, cudaStream_t s)
+{
+    const int64_t warps = (rows * (cols >> 3) + 31) / 32;
+    int64_t grid = (warps + 7) / 8;
+    const int64_t cap = static_cast<int64_t>(sm_count) * 16;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    if (sr)
+        quant_rowwise_kernel<true><<<static_cast<int>(grid), 256, 0, s>>>(
+            x, rows, cols, ld, src, amax_out0, amax_out1, codes, scales, seed, offset,
+            dev_status);
+    else
+        quant_rowwise_kernel<false><<<static_cast<int>(grid), 256, 0, s>>>(
+            x, rows, cols, ld, src, amax_out0, amax_out1, codes, scales, seed, offset,
+            dev_status);
+    return cudaGetLastError();
+}
+
+template <bool ROW, bool COL, bool B2D, bool RHT, bool SR>
+static void launch_tile_t(const TileArgs& a, int grid, cudaStream_t s)
+{
+    quant_tile_kernel<ROW, COL, B2D, RHT, SR><<<grid, 128, 0, s>>>(a);
+}
+
+cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2d, bool rht,
+                              bool sr, int sm_count, cudaStream_t s)
+{
+    const int64_t ntiles = ((a.rows + kTileRows - 1) / kTileRows) *
+                           ((a.cols + kTileCols - 1) / kTileCols);
+    int64_t grid = ntiles;
+    const int64_t cap = static_cast<int64_t>(sm_count) * 16;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    const int g = static_cast<int>(grid);
+    // Supported combinations (the API rejects the others before launching).
+    if (row && col && block2d)            launch_tile_t<true, true, true, false, false>(a, g, s);
+    else if (row && !col && block2d)      launch_tile_t<true, false, true, false, false>(a, g, s);
+    else if (!row && col && block2d)      launch_tile_t<false, true, true, false, false>(a, g, s);
+    else if (row && col && !sr)           launch_tile_t<true, true, false, false, false>(a, g, s);
+    else if (row && col && sr)            launch_tile_t<true, true, false, false, true>(a, g, s);
+    else if (col && rht && sr)            launch_tile_t<false, true, false, true, true>(a, g, s);
+    else if (col && rht && !sr)           launch_tile_t<false, true, false, true, false>(a, g, s);
+    else if (col && !rht && sr)           launch_tile_t<false, true, false, false, true>(a, g, s);
+    else if (col && !rht && !sr)          launch_tile_t<false, true, false, false, false>(a, g, s);
+    else return cudaErrorInvalidValue;
+    return cudaGetLastError();
+}
+
+}  // namespace nvfp4
