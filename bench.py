@@ -72,7 +72,8 @@ def whole_job_rate(units_per_rank: float, world: int, seconds_max: float) -> flo
 # ---- clocks ------------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons with nvidia-smi (every 50 ms) while running.
+    `mark()` opens and closes the window whose samples `summary()` reports."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
@@ -81,8 +82,9 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.device_index = device_index
         self.proc = None
-        self.lines = []
+        self.samples = []  # (host time, csv line)
         self.thread = None
+        self.window = [None, None]
 
     def __enter__(self):
         try:
@@ -92,16 +94,23 @@ class ClockSampler:
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            t0 = time.time()
+            while not self.samples and time.time() - t0 < 10 and self.proc.poll() is None:
+                time.sleep(0.05)  # the first sample marks nvidia-smi as running
         except OSError:
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.samples.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        self.window[0 if which == "start" else 1] = time.time()
 
     def __exit__(self, *exc):
         if self.proc is not None:
+            time.sleep(0.1)
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -111,15 +120,19 @@ class ClockSampler:
                 self.thread.join(timeout=2)
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
+        t0, t1 = self.window
+        lines = [l for t, l in self.samples
+                 if (t0 is None or t >= t0) and (t1 is None or t <= t1 + 0.05)]
+        sm, smax, power, reasons = [], [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 7:
                 continue
             try:
                 sm.append(float(parts[0]))
                 smax.append(float(parts[1]))
+                power.append(float(parts[2]))
             except ValueError:
                 continue
             for name, val in zip(names, parts[3:7]):
@@ -128,7 +141,7 @@ class ClockSampler:
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "power_w_max": max(power), "reasons": sorted(reasons), "samples": len(sm)}
 
 
 # ---- the workload ------------------------------------------------------------------------
@@ -263,23 +276,23 @@ class Step:
 # ---- CPU oracle leg ----------------------------------------------------------------------
 
 def oracle_sample(workload, tokens=128, max_out=512, max_in=4096):
-    """Time the CPU oracle on a bounded sample of the workload: for every linear, the first
-    `tokens` tokens, the first min(O, max_out) out-features and min(I, max_in) in-features;
-    the three GEMMs' operand quantizations and FP64 reference products.  Returns
-    (seconds, GEMM flops of the sample, threads used)."""
+    """Time the CPU oracle on a bounded sample of the workload: for every linear, a
+    `tokens` x min(I, max_in) activation, a min(O, max_out) x min(I, max_in) weight and a
+    `tokens` x min(O, max_out) gradient drawn with the workload's generators and seed; the
+    timed part is the three GEMMs' operand quantizations and FP64 reference products.
+    Returns (seconds, GEMM flops of the sample, threads used)."""
     import oracle
+    inputs = []
+    for li, lin in enumerate(workload.linears):
+        small = synth.Linear(lin.name, tokens, min(lin.I, max_in), min(lin.O, max_out))
+        inputs.append(synth.linear_inputs(small, workload.seed, layer_index=li))
+    mask = oracle.sign_mask_from_seed(workload.seed)
     flops = 0
     t0 = time.perf_counter()
-    for li, lin in enumerate(workload.linears):
-        X, W, dY = synth.linear_inputs(lin, workload.seed, layer_index=li)
-        Ts, Is, Os = tokens, min(lin.I, max_in), min(lin.O, max_out)
-        Xs = np.ascontiguousarray(X[:Ts, :Is])
-        Ws = np.ascontiguousarray(W[:Os, :Is])
-        dYs = np.ascontiguousarray(dY[:Ts, :Os])
-        mask = oracle.sign_mask_from_seed(workload.seed)
-        for qa, qb in (oracle.fprop_operands(Xs, Ws),
-                       oracle.dgrad_operands(dYs, Ws, workload.seed, 0),
-                       oracle.wgrad_operands(dYs, Xs, mask, workload.seed, 0)):
+    for X, W, dY in inputs:
+        for qa, qb in (oracle.fprop_operands(X, W),
+                       oracle.dgrad_operands(dY, W, workload.seed, 0),
+                       oracle.wgrad_operands(dY, X, mask, workload.seed, 0)):
             oracle.gemm_ref(qa, qb)
             flops += 2 * qa.rows * qb.rows * qa.cols
     secs = time.perf_counter() - t0
@@ -292,11 +305,12 @@ def oracle_sample(workload, tokens=128, max_out=512, max_in=4096):
 
 
 def cpu_baseline(workload):
-    secs, flops, threads = oracle_sample(workload)
+    secs, flops, threads = oracle_sample(workload, tokens=1024, max_out=2048, max_in=5120)
     return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "sample": "per linear: first 128 tokens, first min(O,512) out- and min(I,4096) "
-                      "in-features; fprop/dgrad/wgrad operand quantization (C oracle) + FP64 "
-                      "reference GEMM (numpy matmul of dequantized operands)",
+            "sample": "per linear: 1024 tokens x min(O,2048) out- x min(I,5120) in-features drawn "
+                      "with the workload's generators; fprop/dgrad/wgrad operand quantization "
+                      "(C oracle, 1 thread) + FP64 reference GEMMs (numpy matmul of the "
+                      "dequantized operands)",
             "seconds": secs}
 
 
@@ -306,15 +320,16 @@ def run_reference(args):
         return 0
     wl = synth.mlp_12b()
     for _ in range(args.warmup):
-        oracle_sample(wl, tokens=64, max_out=256, max_in=2048)
+        oracle_sample(wl, tokens=128, max_out=512, max_in=4096)
     times, flops, threads = [], 0, 1
     for _ in range(args.steps):
-        secs, flops, threads = oracle_sample(wl, tokens=64, max_out=256, max_in=2048)
+        secs, flops, threads = oracle_sample(wl, tokens=128, max_out=512, max_in=4096)
         times.append(secs)
     total = sum(times)
     value = flops * len(times) / total / 1e12
-    sample = ("per linear: first 64 tokens, first min(O,256) out- and min(I,2048) in-features; "
-              "operand quantization (C oracle) + FP64 reference GEMMs")
+    sample = ("per linear: 128 tokens x min(O,512) out- x min(I,4096) in-features drawn with "
+              "the workload's generators; operand quantization (C oracle, 1 thread) + FP64 "
+              "reference GEMMs (numpy matmul)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
@@ -347,17 +362,17 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    for _ in range(args.warmup):
-        step.run()
-    torch.cuda.synchronize()
-    st = int(step.dev_status.item())
-    if st != 0:
-        raise RuntimeError(f"device status {st} after warm-up")
-
     events = {"gemm": [], "quant": []}
     with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        for _ in range(args.warmup):
+            step.run()
+        torch.cuda.synchronize()
+        st = int(step.dev_status.item())
+        if st != 0:
+            raise RuntimeError(f"device status {st} after warm-up")
         barrier()
         torch.cuda.synchronize()
+        clocks.mark("start")
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record()
@@ -365,6 +380,7 @@ def run_ours(args):
             step.run(events)
         t1.record()
         torch.cuda.synchronize()
+        clocks.mark("end")
         barrier()
     ms_local = t0.elapsed_time(t1) / args.steps
     ms = max_over_ranks(ms_local, device)
@@ -441,18 +457,71 @@ def run_ours(args):
     return 0 if st == 0 else 1
 
 
+def run_kernel_case(args):
+    """One kernel family alone, at the MLP workload's shapes, for profiling: warm-up launches,
+    then `steps` launches bracketed by CUDA events.  Prints a JSON line (not a bench value)."""
+    import torch
+    from nvfp4_bit_quantized_03_b200 import binding as B
+    peaks = _peaks()
+    T, D, F = 8192, 5120, 20480
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ws = torch.empty((B.workspace_bytes(1 << 14, 1 << 14),), dtype=torch.uint8, device=dev)
+    if args.kernel == "gemm":
+        X = torch.from_numpy(synth.activations((T, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
+        W = torch.from_numpy(synth.weights((F, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
+        qa, _ = B.quantize(X, B.ROWWISE, workspace=ws)
+        qb, _ = B.quantize(W, B.ROWWISE | B.BLOCK2D, workspace=ws)
+        out = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
+        fn = lambda: B.gemm(qa, qb, out=out)  # noqa: E731
+        work, unit, peak = 2 * T * D * F / 1e12, "TFLOP/s", peaks["bf16_tflops"] * FP4_OVER_BF16
+        shape = f"M={T} N={F} K={D}, bf16 out"
+    else:
+        x = torch.from_numpy(synth.gradients((T, F), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
+        n = T * F
+        if args.kernel == "rowwise":
+            q = B.QuantizedTensor(T, F, dev)
+            fn = lambda: B.quantize(x, B.ROWWISE | B.SR, seed=1, out_row=q, workspace=ws)  # noqa: E731
+        elif args.kernel == "tile2d":
+            q = B.QuantizedTensor(F, T, dev)
+            fn = lambda: B.quantize(x, B.COLWISE | B.BLOCK2D, out_col=q, workspace=ws)  # noqa: E731
+        else:
+            q = B.QuantizedTensor(F, T, dev)
+            fn = lambda: B.rht_quantize(x, 0x5A3C, B.SR, seed=1, out_col=q, workspace=ws)  # noqa: E731
+        work, unit, peak = n * (4 + 0.5 + 1 / 16) / 1e9, "GB/s", peaks["hbm_gbs"]
+        shape = f"{T} x {F} bf16, amax pass + quantize pass"
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    rate = work / (ms / 1e3)
+    print(json.dumps({"kernel_case": args.kernel, "shape": shape, "ms_per_launch": ms,
+                      "achieved": rate, "unit": unit, "peak": peak, "frac": rate / peak}),
+          flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["gemm", "rowwise", "tile2d", "rht"], default=None,
+                    help="time one kernel family alone at the workload's shapes (profiling)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
+    if args.kernel:
+        return run_kernel_case(args)
     return run_ours(args)
 
 

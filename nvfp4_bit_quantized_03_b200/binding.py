@@ -146,6 +146,14 @@ class QuantizedTensor:
                        self.rows, self.cols)
 
 
+def _dtype_code(dtype):
+    if dtype == torch.float32:
+        return OUT_F32
+    if dtype == torch.bfloat16:
+        return OUT_BF16
+    raise TypeError(f"unsupported output dtype {dtype}")
+
+
 def _workspace(nbytes, device):
     if nbytes == 0:
         return None
@@ -190,11 +198,21 @@ def rht_quantize(x, sign_mask, flags=0, seed=0, offset=0, out_col=None, workspac
     return out_col
 
 
+def _check_out(out, rows, cols, what):
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"{what}: output must be float32 or bfloat16, got {out.dtype}")
+    if tuple(out.shape) != (rows, cols) or out.stride(1) != 1 or not out.is_cuda:
+        raise ValueError(f"{what}: output must be a CUDA [{rows} x {cols}] tensor with unit "
+                         f"column stride, got {tuple(out.shape)} strides {out.stride()}")
+
+
 def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None):
-    """nvfp4_gemm: D = A . B^T (A, B QuantizedTensor)."""
-    d_dtype = OUT_F32 if out_dtype == torch.float32 else OUT_BF16
+    """nvfp4_gemm: D = A . B^T (A, B QuantizedTensor).  The output type is out.dtype when
+    `out` is given, else `out_dtype`."""
     if out is None:
         out = torch.empty((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
+    _check_out(out, A.rows, B.rows, "nvfp4_gemm")
+    d_dtype = _dtype_code(out.dtype)
     oa, ob = A.operand(), B.operand()
     st = lib().nvfp4_gemm(ctypes.byref(oa), ctypes.byref(ob), _ptr(out), d_dtype, out.stride(0),
                           _ptr(dev_status), _stream(stream))
@@ -202,8 +220,6 @@ def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None):
     return out
 
 
-def _dtype_code(dtype):
-    return OUT_F32 if dtype == torch.float32 else OUT_BF16
 
 
 def linear_fprop(X, W, out=None, out_dtype=torch.float32, workspace=None, dev_status=None,
@@ -212,6 +228,7 @@ def linear_fprop(X, W, out=None, out_dtype=torch.float32, workspace=None, dev_st
     O = W.shape[0]
     if out is None:
         out = torch.empty((T, O), dtype=out_dtype, device=X.device)
+    _check_out(out, T, O, "nvfp4_linear_fprop")
     if workspace is None:
         workspace = _workspace(linear_workspace_bytes(T, I, O), X.device)
     st = lib().nvfp4_linear_fprop(_ptr(X), _ptr(W), T, I, O, _ptr(out), _dtype_code(out.dtype),
@@ -226,6 +243,7 @@ def linear_dgrad(dY, W, seed, offset, out=None, out_dtype=torch.float32, workspa
     I = W.shape[1]
     if out is None:
         out = torch.empty((T, I), dtype=out_dtype, device=dY.device)
+    _check_out(out, T, I, "nvfp4_linear_dgrad")
     if workspace is None:
         workspace = _workspace(linear_workspace_bytes(T, I, O), dY.device)
     st = lib().nvfp4_linear_dgrad(_ptr(dY), _ptr(W), T, I, O, seed, offset, _ptr(out),
@@ -241,6 +259,7 @@ def linear_wgrad(dY, X, sign_mask, seed, offset, out=None, out_dtype=torch.float
     I = X.shape[1]
     if out is None:
         out = torch.empty((O, I), dtype=out_dtype, device=dY.device)
+    _check_out(out, O, I, "nvfp4_linear_wgrad")
     if workspace is None:
         workspace = _workspace(linear_workspace_bytes(T, I, O), dY.device)
     st = lib().nvfp4_linear_wgrad(_ptr(dY), _ptr(X), T, I, O, sign_mask, seed, offset, _ptr(out),

@@ -175,3 +175,14 @@ def test_valid_call_without_gpu_fails_cleanly():
     st = L.nvfp4_quantize(ctypes.c_void_p(0x1000), 256, 512, 512, B.ROWWISE, 0, 0,
                           ctypes.byref(out), None, ctypes.c_void_p(0x8000), None, None)
     assert st in (B.ERR_CUDA, B.ERR_DEVICE)
+
+
+def test_binding_rejects_bad_output_tensors_before_calling():
+    A = B.QuantizedTensor(128, 256, device="cpu")
+    Bq = B.QuantizedTensor(256, 256, device="cpu")
+    with pytest.raises(TypeError):
+        B.gemm(A, Bq, out=torch.empty((128, 256), dtype=torch.float16))
+    with pytest.raises(ValueError):
+        B.gemm(A, Bq, out=torch.empty((128, 200), dtype=torch.float32))
+    with pytest.raises(ValueError):  # host tensor
+        B.gemm(A, Bq, out=torch.empty((128, 256), dtype=torch.bfloat16))
