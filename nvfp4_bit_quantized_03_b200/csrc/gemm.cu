@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // ---------------- TMA producer ----------------
         int stage = 0;
         uint32_t phase = 0;
-        uint32_t issued[STAGES] = {0, 0, 0, 0};
+        uint32_t issued[STAGES] = {};
         bool ok = true;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
             int tm, tn;
