@@ -214,6 +214,28 @@ nvfp4_status nvfp4_linear_wgrad(const void* dY, const void* X, int64_t T, int64_
                                 uint16_t sign_mask, uint64_t seed, uint64_t offset, void* dW,
                                 int dw_dtype, void* workspace, int* dev_status, void* stream);
 
+/*
+ * nvfp4_quantize without a caller workspace, for callers that cannot allocate device memory
+ * where they quantize (a host framework that owns all device memory through its own
+ * fixed arena, or a latency-critical loop that must not enter cudaMalloc / cudaFree, which may
+ * block or synchronize the device).  The pages have no counterpart to this call: it is a
+ * deployment convenience of this library.
+ *
+ * Same arguments, rules and results as nvfp4_quantize, minus `workspace`: the partial maxima
+ * of the amax pass live in a file-scope device array of NVFP4_NOALLOC_MAX_PARTIALS 32-bit slots
+ * (8 KB per GPU that loads the library, held until the process exits).  The call allocates
+ * nothing.  The first call on each device looks up the array's address; make it before any
+ * stream capture begins.  Calls share the array: calls whose kernels overlap on the GPU
+ * (several streams or host threads on one device) race and may give wrong results; calls on
+ * one stream are safe.  A shape needing more slots than the array holds returns
+ * NVFP4_ERR_SHAPE.
+ */
+#define NVFP4_NOALLOC_MAX_PARTIALS 2048
+nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                    unsigned flags, uint64_t seed, uint64_t offset,
+                                    const nvfp4_operand* out_row, const nvfp4_operand* out_col,
+                                    int* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -21,6 +21,7 @@ UNITS = {
     "api.cu": [],
     "quantize.cu": ["-fmad=false"],
     "gemm.cu": [],
+    "noalloc.cu": [],
 }
 
 
