@@ -4,19 +4,23 @@
 // tecnico section 2, "Formato NVFP4": E2M1 operands with one E4M3 scale per 16 elements and
 // an FP32 scale per tensor, multiplied natively by Blackwell tensor cores.
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles):
+// Design (one CTA per SM, persistent over 128 x 256 output tiles, 22 warps):
 //   warp 0      TMA producer: per 256-wide K block, the A (128 x 128 B) and B (256 x 128 B)
 //               code tiles with 128-byte swizzle, plus the block scales (contiguous 512-byte
-//               tiles of the MMA scale layout) by bulk copies; a 4-stage shared-memory ring
+//               tiles of the MMA scale layout) by bulk copies; a 3-stage shared-memory ring
 //               guarded by mbarriers.
-//   warp 1      TMEM owner and MMA issuer (one thread): copies each stage's scales
-//               shared -> tensor memory (tcgen05.cp 32x128b.warpx4, into a per-stage
-//               column range) and issues tcgen05.mma kind::mxf4nvf4 (M 128, N 256, K 64,
-//               FP32 accumulation in TMEM), then commits the stage back to the producer.
-//   warps 2-9   epilogue: each warp drains one 32-lane quarter x 128 columns of the
+//   warps 2-5   scale stagers, one per 32-lane quarter of tensor memory: move each stage's
+//               scales shared -> registers -> tensor memory (ld.shared + tcgen05.st, into a
+//               per-stage column range), so the tensor pipe never spends time on scale copies.
+//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::mxf4nvf4 (M 128,
+//               N 256, K 64, FP32 accumulation in TMEM), then commits the stage back to the
+//               producer.
+//   warps 6-21  epilogue: each warp drains one 32-lane quarter x 64 columns of the
 //               accumulator into registers (tcgen05.ld), releases the accumulator so the
 //               next tile's MMAs start at once, then scales by 1 / (S_enc,A S_enc,B) and
-//               stores FP32 or bf16 rows while the next tile computes.
+//               writes FP32 or bf16 rows through a 64-byte-swizzled shared-memory staging
+//               buffer with TMA bulk tensor stores (whole 64-byte row segments, clipped at the
+//               matrix edge) while the next tile computes.
 // Every wait on an mbarrier is bounded in time; on expiry the kernel records
 // NVFP4_DEVSTAT_TIMEOUT, drains its in-flight copies and MMAs (again with a limit), frees
 // its tensor memory and returns.
@@ -38,21 +42,26 @@ constexpr int BM = 128;                 // tile rows (A rows, TMEM lanes)
 constexpr int BN = 256;                 // tile columns (B rows, accumulator columns)
 constexpr int BK = 256;                 // K elements per pipeline stage (128 bytes per row)
 constexpr int MMA_K = 64;               // K per tcgen05.mma of kind::mxf4nvf4
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BK / 2;    // 16 KB
 constexpr int B_BYTES = BN * BK / 2;    // 32 KB
 constexpr int SF_TILE = 512;            // 128 rows x 4 blocks of scales
 constexpr int SFA_BYTES = (BM / 128) * (BK / MMA_K) * SF_TILE;  // 2 KB
 constexpr int SFB_BYTES = (BN / 128) * (BK / MMA_K) * SF_TILE;  // 4 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int NUM_SF_WARPS = 4;         // one per 32-lane quarter of tensor memory
+constexpr int NUM_EPI_WARPS = 16;       // four per lane quarter, 64 accumulator columns each
+constexpr int FIRST_SF_WARP = 2;
+constexpr int FIRST_EPI_WARP = FIRST_SF_WARP + NUM_SF_WARPS;
+constexpr int THREADS = 32 * (FIRST_EPI_WARP + NUM_EPI_WARPS);
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;              // accumulator: columns [0, 256)
 constexpr int SF_COL = BN;              // scales: 48 columns per stage from column 256
 constexpr int SF_COLS_PER_STAGE = (BK / MMA_K) * (4 + 8);
-constexpr int BAR_BYTES = 128;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + BAR_BYTES + 1024;
+constexpr int STAGING_BYTES = 2048;     // per epilogue warp: 32 rows x 64 bytes of output
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NUM_EPI_WARPS * STAGING_BYTES + BAR_BYTES + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait
 constexpr int kDevTimeoutBit = 2;       // NVFP4_DEVSTAT_TIMEOUT
 
@@ -155,6 +164,20 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
         : "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x,
+                                             int32_t y)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(src)
+        : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 // ---- tcgen05 -----------------------------------------------------------------------------
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -167,19 +190,32 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr)
            (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
            (static_cast<uint64_t>(2) << 61);
 }
-// Descriptor of one 512-byte scale tile for tcgen05.cp: no swizzle, 32 rows of 16 bytes,
-// 8-row core matrices 128 bytes apart, a single 16-byte column.
-__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr)
+// Register -> tensor memory stores of one warp's 32 lanes: 16 or 32 consecutive columns.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v)
 {
-    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) |
-           (static_cast<uint64_t>(128 >> 4) << 32) | (static_cast<uint64_t>(1) << 46);
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15])
+        : "memory");
 }
-
-__device__ __forceinline__ void tmem_copy_sf(uint32_t taddr, uint64_t sdesc)
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v)
 {
-    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-                 : "memory");
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(
+            taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
 }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc,
                                          uint32_t sfa, uint32_t sfb, uint32_t accumulate)
@@ -238,17 +274,74 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
     tn = local / gsz;
 }
 
+// One epilogue warp's 32 x 64 slice of the tile (row `lane`, values v[0..63] in FP32 bits) to
+// global memory: scaled by alpha, converted, written as 32 x 64-byte boxes into the warp's
+// staging buffer and sent with TMA bulk tensor stores (bf16: 2 boxes of 32 columns; FP32: 4
+// boxes of 16).  Row `lane` of a box sits at lane * 64 with its four 16-byte chunks permuted
+// by the 64-byte swizzle (chunk c at c ^ ((row / 2) % 4)), which the tensor map undoes.
+template <bool BF16>
+__device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint32_t stage_buf,
+                                            int lane, const CUtensorMap* tmap_d, int n0, int y,
+                                            int M, int N)
+{
+    constexpr int COLS = BF16 ? 32 : 16;  // columns per 64-byte box row
+    const uint32_t row_base = stage_buf + 64 * lane;
+    const uint32_t swz = (lane >> 1) & 3;
+#pragma unroll
+    for (int r = 0; r < 64 / COLS; ++r) {
+        if (lane == 0) bulk_wait_read();  // the previous box has left the buffer
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            uint32_t o[4];
+            if (BF16) {
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    const int j = r * 32 + c * 8 + 2 * h;
+                    const __nv_bfloat162 b2 =
+                        __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j]), alpha),
+                                              __fmul_rn(__uint_as_float(v[j + 1]), alpha));
+                    o[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+            } else {
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                    o[h] = __float_as_uint(__fmul_rn(__uint_as_float(v[r * 16 + c * 4 + h]), alpha));
+            }
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_base + 16 * (c ^ swz)),
+                         "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
+                         : "memory");
+        }
+        fence_async_smem();
+        __syncwarp();
+        const int x = n0 + r * COLS;
+        if (lane == 0 && y < M && x < N) tma_store_2d(tmap_d, stage_buf, x, y);
+    }
+}
+
+// Shared-memory barrier slots.
+constexpr int BAR_FULL = 0;                 // [STAGES] TMA bytes of a stage landed
+constexpr int BAR_EMPTY = BAR_FULL + STAGES;    // [STAGES] the stage's MMAs completed
+constexpr int BAR_SF = BAR_EMPTY + STAGES;      // [STAGES] the stage's scales are in TMEM
+constexpr int BAR_ACC_FULL = BAR_SF + STAGES;   // the tile's accumulator is complete
+constexpr int BAR_ACC_EMPTY = BAR_ACC_FULL + 1; // the epilogue drained the accumulator
+constexpr int BAR_DRAIN = BAR_ACC_EMPTY + 1;    // teardown after an abort
+constexpr int NUM_BARS = BAR_DRAIN + 1;
+static_assert(NUM_BARS * 8 + 16 <= BAR_BYTES, "barrier area");
+
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                     const __grid_constant__ CUtensorMap tmap_b, const Params p)
+                     const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ CUtensorMap tmap_d, const Params p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    // bars[0..3] full, [4..7] empty, [8] acc_full, [9] acc_empty, [10] drain
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 12);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 13);
+    uint8_t* staging = smem + STAGES * STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(staging + NUM_EPI_WARPS * STAGING_BYTES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles_m = (p.M + BM - 1) / BM, tiles_n = (p.N + BN - 1) / BN;
@@ -260,16 +353,18 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&bars[s]), 1);
-            mbar_init(smem_u32(&bars[STAGES + s]), 1);
+            mbar_init(bar(BAR_FULL + s), 1);
+            mbar_init(bar(BAR_EMPTY + s), 1);
+            mbar_init(bar(BAR_SF + s), NUM_SF_WARPS);
         }
-        mbar_init(smem_u32(&bars[8]), 1);
-        mbar_init(smem_u32(&bars[9]), NUM_EPI_WARPS);
-        mbar_init(smem_u32(&bars[10]), 1);
+        mbar_init(bar(BAR_ACC_FULL), 1);
+        mbar_init(bar(BAR_ACC_EMPTY), NUM_EPI_WARPS);
+        mbar_init(bar(BAR_DRAIN), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_d)) : "memory");
     }
     if (warp == 1) {
         __syncwarp();
@@ -294,15 +389,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             int tm, tn;
             tile_coords(t, tiles_m, tiles_n, tm, tn);
             for (int kb = 0; kb < num_kb; ++kb) {
-                if (!wait_bounded(smem_u32(&bars[STAGES + stage]), phase ^ 1, abort_flag,
-                                  p.dev_status)) {
+                if (!wait_bounded(bar(BAR_EMPTY + stage), phase ^ 1, abort_flag, p.dev_status)) {
                     ok = false;
                     break;
                 }
                 const int natoms = min(BK / MMA_K, sf_groups - kb * (BK / MMA_K));
                 const bool b2 = (2 * tn + 1) < sfb_row_tiles;
                 const uint32_t sf_bytes = natoms * SF_TILE * (b2 ? 3u : 2u);
-                const uint32_t full = smem_u32(&bars[stage]);
+                const uint32_t full = bar(BAR_FULL + stage);
                 uint8_t* st = smem + stage * STAGE_BYTES;
                 mbar_expect_tx(full, A_BYTES + B_BYTES + sf_bytes);
                 tma_load_2d(smem_u32(st), &tmap_a, kb * (BK / 2), tm * BM, full);
@@ -326,7 +420,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             // Let every copy already issued land before the CTA can exit.
             for (int s = 0; s < STAGES; ++s)
                 if (issued[s])
-                    wait_bounded(smem_u32(&bars[s]), (issued[s] - 1) & 1, abort_flag, nullptr, true);
+                    wait_bounded(bar(BAR_FULL + s), (issued[s] - 1) & 1, abort_flag, nullptr, true);
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer ----------------
@@ -335,50 +429,104 @@ __global__ void __launch_bounds__(THREADS, 1)
         bool ok = true, any = false;
         int it = 0;
         for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
-            if (!wait_bounded(smem_u32(&bars[9]), (it & 1) ^ 1, abort_flag, p.dev_status)) {
+            if (!wait_bounded(bar(BAR_ACC_EMPTY), (it & 1) ^ 1, abort_flag, p.dev_status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             for (int kb = 0; kb < num_kb; ++kb) {
-                if (!wait_bounded(smem_u32(&bars[stage]), phase, abort_flag, p.dev_status)) {
+                // the stage's codes are in shared memory and its scales in tensor memory
+                if (!wait_bounded(bar(BAR_SF + stage), phase, abort_flag, p.dev_status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint8_t* st = smem + stage * STAGE_BYTES;
                 const uint32_t a0 = smem_u32(st), b0 = smem_u32(st + A_BYTES);
-                const uint32_t sfa0 = smem_u32(st + A_BYTES + B_BYTES);
-                const uint32_t sfb0 = sfa0 + SFA_BYTES;
                 const uint32_t tcol = tmem_base + SF_COL + stage * SF_COLS_PER_STAGE;
                 const int nk = min(BK / MMA_K, k_steps_total - kb * (BK / MMA_K));
                 for (int k = 0; k < nk; ++k) {
-                    tmem_copy_sf(tcol + 4 * k, desc_sf(sfa0 + k * SF_TILE));
-                    tmem_copy_sf(tcol + 16 + 8 * k, desc_sf(sfb0 + k * SF_TILE));
-                    tmem_copy_sf(tcol + 16 + 8 * k + 4, desc_sf(sfb0 + SFB_BYTES / 2 + k * SF_TILE));
-                }
-                for (int k = 0; k < nk; ++k) {
-                    // K step k = 64 elements = 32 bytes into the 128-byte swizzled rows
+                    // K step k = 64 elements = 32 bytes into the 128-byte swizzled rows; its
+                    // scales: A in columns tcol + 4k, B in tcol + 16 + 8k
                     mma_nvf4(tmem_base + ACC_COL, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k),
                              tcol + 4 * k, tcol + 16 + 8 * k, (kb | k) != 0 ? 1u : 0u);
                 }
                 any = true;
-                mma_commit(smem_u32(&bars[STAGES + stage]));
+                mma_commit(bar(BAR_EMPTY + stage));
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
-            if (ok) mma_commit(smem_u32(&bars[8]));
+            if (ok) mma_commit(bar(BAR_ACC_FULL));
         }
         if (!ok && any) {
-            mma_commit(smem_u32(&bars[10]));
-            wait_bounded(smem_u32(&bars[10]), 0, abort_flag, nullptr, true);
+            mma_commit(bar(BAR_DRAIN));
+            wait_bounded(bar(BAR_DRAIN), 0, abort_flag, nullptr, true);
         }
-    } else if (warp >= 2) {
+    } else if (warp >= FIRST_SF_WARP && warp < FIRST_SF_WARP + NUM_SF_WARPS) {
+        // ---------------- scale stagers ----------------
+        // Tensor-memory layout the block-scaled MMA reads: row r's four E4M3 scales of one
+        // K step sit in lane r % 32 of every lane quarter, column r / 32.  Byte 16 l of a
+        // 512-byte scale tile holds exactly those 4 columns for rows l, l + 32, l + 64,
+        // l + 96, so lane l of each quarter's warp loads 16 bytes per tile and stores them.
+        const int q = warp & 3;
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                bool ready = lane == 0 ? wait_bounded(bar(BAR_FULL + stage), phase, abort_flag,
+                                                      p.dev_status)
+                                       : false;
+                ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
+                if (!ready) {
+                    ok = false;
+                    break;
+                }
+                __syncwarp();
+                const uint8_t* sf = smem + stage * STAGE_BYTES + A_BYTES + B_BYTES;
+                uint32_t ra[16], rb[32];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const uint4 v = *reinterpret_cast<const uint4*>(sf + k * SF_TILE + 16 * lane);
+                    ra[4 * k] = v.x;
+                    ra[4 * k + 1] = v.y;
+                    ra[4 * k + 2] = v.z;
+                    ra[4 * k + 3] = v.w;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 v = *reinterpret_cast<const uint4*>(
+                            sf + SFA_BYTES + h * (SFB_BYTES / 2) + k * SF_TILE + 16 * lane);
+                        const int c = 4 * (2 * k + h);
+                        rb[c] = v.x;
+                        rb[c + 1] = v.y;
+                        rb[c + 2] = v.z;
+                        rb[c + 3] = v.w;
+                    }
+                }
+                const uint32_t taddr = tmem_base + SF_COL + stage * SF_COLS_PER_STAGE +
+                                       (static_cast<uint32_t>(32 * q) << 16);
+                tmem_st16(taddr, ra);       // A: columns 4k + j
+                tmem_st32(taddr + 16, rb);  // B: columns 16 + 8k + 4h + j
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(BAR_SF + stage));
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
+        }
+    } else if (warp >= FIRST_EPI_WARP) {
         // ---------------- epilogue ----------------
-        const int q = warp & 3;              // TMEM lane quarter this warp may access
-        const int half = (warp - 2) >> 2;    // accumulator columns [128 half, 128 half + 128)
+        const int q = warp & 3;                         // TMEM lane quarter this warp may access
+        const int chunk = (warp - FIRST_EPI_WARP) >> 2; // accumulator columns [64 chunk, +64)
+        const uint32_t stage_buf = smem_u32(staging + (warp - FIRST_EPI_WARP) * STAGING_BYTES);
         const float aa = *p.amax_a, ab = *p.amax_b;
         const bool finite = (aa < INFINITY) && (ab < INFINITY) && aa >= 0.0f && ab >= 0.0f;
         const float alpha =
@@ -386,63 +534,33 @@ __global__ void __launch_bounds__(THREADS, 1)
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
             // one lane waits, so the whole warp takes the same branch into tcgen05.ld
-            bool ready = lane == 0 ? wait_bounded(smem_u32(&bars[8]), it & 1, abort_flag,
+            bool ready = lane == 0 ? wait_bounded(bar(BAR_ACC_FULL), it & 1, abort_flag,
                                                   p.dev_status)
                                    : false;
             ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
             if (!ready) break;
             __syncwarp();
             tc_fence_after();
-            uint32_t v[128];
+            uint32_t v[64];
             const uint32_t taddr = tmem_base + ACC_COL + (static_cast<uint32_t>(32 * q) << 16) +
-                                   128 * half;
+                                   64 * chunk;
             tmem_ld32(taddr, v);
             tmem_ld32(taddr + 32, v + 32);
-            tmem_ld32(taddr + 64, v + 64);
-            tmem_ld32(taddr + 96, v + 96);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&bars[9]));
+            if (lane == 0) mbar_arrive(bar(BAR_ACC_EMPTY));
 
             int tm, tn;
             tile_coords(t, tiles_m, tiles_n, tm, tn);
-            const int m = tm * BM + 32 * q + lane;
-            const int n0 = tn * BN + 128 * half;
-            if (m < p.M) {
-                if (p.out_bf16) {
-                    __nv_bfloat16* row = reinterpret_cast<__nv_bfloat16*>(p.D) + m * p.ldd;
-#pragma unroll
-                    for (int j = 0; j < 128; j += 8) {
-                        if (n0 + j < p.N) {
-                            uint4 o;
-                            uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                            for (int h = 0; h < 4; ++h) {
-                                const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                                    __fmul_rn(__uint_as_float(v[j + 2 * h]), alpha),
-                                    __fmul_rn(__uint_as_float(v[j + 2 * h + 1]), alpha));
-                                ow[h] = *reinterpret_cast<const uint32_t*>(&b2);
-                            }
-                            *reinterpret_cast<uint4*>(row + n0 + j) = o;
-                        }
-                    }
-                } else {
-                    float* row = reinterpret_cast<float*>(p.D) + m * p.ldd;
-#pragma unroll
-                    for (int j = 0; j < 128; j += 4) {
-                        if (n0 + j < p.N) {
-                            float4 o;
-                            o.x = __fmul_rn(__uint_as_float(v[j]), alpha);
-                            o.y = __fmul_rn(__uint_as_float(v[j + 1]), alpha);
-                            o.z = __fmul_rn(__uint_as_float(v[j + 2]), alpha);
-                            o.w = __fmul_rn(__uint_as_float(v[j + 3]), alpha);
-                            *reinterpret_cast<float4*>(row + n0 + j) = o;
-                        }
-                    }
-                }
-            }
+            const int y = tm * BM + 32 * q;       // first output row of this warp's slice
+            const int n0 = tn * BN + 64 * chunk;  // first output column
+            if (p.out_bf16)
+                store_slice<true>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
+            else
+                store_slice<false>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
         }
+        if (lane == 0) bulk_wait_all();
     }
 
     tc_fence_before();
@@ -488,6 +606,22 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2D map over D (rows x N elements, row stride ldd), boxes of 32 rows x 64 bytes with
+// 64-byte swizzle, for the epilogue's bulk tensor stores.
+bool make_output_map(CUtensorMap* map, void* D, int64_t M, int64_t N, int64_t ldd, bool bf16)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int64_t esize = bf16 ? 2 : 4;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldd * esize)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / esize), 32};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, D,
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
@@ -501,8 +635,9 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
-    CUtensorMap ma, mb;
-    if (!make_codes_map(&ma, g.a_codes, g.M, g.K, BM) || !make_codes_map(&mb, g.b_codes, g.N, g.K, BN))
+    CUtensorMap ma, mb, md;
+    if (!make_codes_map(&ma, g.a_codes, g.M, g.K, BM) || !make_codes_map(&mb, g.b_codes, g.N, g.K, BN) ||
+        !make_output_map(&md, g.D, g.M, g.N, g.ldd, g.out_bf16 != 0))
         return cudaErrorInvalidValue;
     Params p;
     p.sfa = g.a_scales;
@@ -518,7 +653,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     p.dev_status = g.dev_status;
     const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < sm_count ? tiles : sm_count);
-    gemm_nvf4_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mb, p);
+    gemm_nvf4_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mb, md, p);
     return cudaGetLastError();
 }
 
