@@ -54,12 +54,13 @@ struct Philox {
         uint32_t a = k0, b = k1;
 #pragma unroll
         for (int i = 0; i < 10; ++i) {
-            const uint32_t lo0 = c0 * 0xD2511F53u, hi0 = __umulhi(c0, 0xD2511F53u);
-            const uint32_t lo1 = c2 * 0xCD9E8D57u, hi1 = __umulhi(c2, 0xCD9E8D57u);
-            c0 = hi1 ^ c1 ^ a;
-            c1 = lo1;
-            c2 = hi0 ^ c3 ^ b;
-            c3 = lo0;
+            // one 32 x 32 -> 64-bit product per multiplier gives both halves
+            const uint64_t p0 = static_cast<uint64_t>(c0) * 0xD2511F53u;
+            const uint64_t p1 = static_cast<uint64_t>(c2) * 0xCD9E8D57u;
+            c0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ a;
+            c1 = static_cast<uint32_t>(p1);
+            c2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ b;
+            c3 = static_cast<uint32_t>(p0);
             a += 0x9E3779B9u;
             b += 0xBB67AE85u;
         }
@@ -142,25 +143,22 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi)
 
 // Stochastic rounding of v to the E2M1 grid with the 16-bit random integer r16: the
 // magnitude goes up to the next grid point iff r16 < p * 65536, p the position of |v|
-// between its grid neighbours.  The grid spacing is 0.5 below 2, 1 below 4 and 2 below 6,
-// so t = |v| / spacing is exact, p = t - floor(t) and the result (floor(t) + up) * spacing
-// is a grid point; it is encoded exactly by the round-to-nearest conversion.
+// between its grid neighbours.  The grid spacing is 0.5 below 2, 1 below 4 and 2 from 4 on,
+// so t = |v| / spacing is exact and p = frac(t).  For integers, r16 < p * 65536 holds iff
+// r16 < ceil(p * 65536) = ceil(t * 65536) - floor(t) * 65536; with xi = ceil(t * 65536) (an
+// exact conversion, t * 65536 being an exact FP32 product) the rounded grid index is
+// (xi >> 16) + (r16 < (xi & 0xFFFF)) -- when the fraction rounds up to a whole 65536 the carry
+// is already in xi >> 16 and the comparison is false.  The result index * spacing is a grid
+// point (anything from 6 up saturates to 6 in the conversion) and keeps the sign of v.
 __device__ __forceinline__ float e2m1_sr_value(float v, uint32_t r16)
 {
     const float a = fabsf(v);
-    float q;
-    if (!(a < 6.0f)) {
-        q = 6.0f;
-    } else {
-        const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-        const float inv = a < 2.0f ? 2.0f : (a < 4.0f ? 1.0f : 0.5f);
-        const float t = __fmul_rn(a, inv);
-        const float f = floorf(t);
-        const float p = __fsub_rn(t, f);
-        const bool up = static_cast<float>(r16) < __fmul_rn(p, 65536.0f);
-        q = __fmul_rn(up ? __fadd_rn(f, 1.0f) : f, step);
-    }
-    return copysignf(q, v);
+    const float c = a < 2.0f ? 131072.0f : (a < 4.0f ? 65536.0f : 32768.0f);  // 65536 / spacing
+    const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
+    uint32_t xi;
+    asm("cvt.rpi.sat.u32.f32 %0, %1;" : "=r"(xi) : "f"(__fmul_rn(a, c)));
+    const uint32_t idx = (xi >> 16) + (r16 < (xi & 0xFFFFu) ? 1u : 0u);
+    return copysignf(__fmul_rn(__uint2float_rn(idx), step), v);
 }
 
 // ---- random Hadamard transform ----------------------------------------------------------

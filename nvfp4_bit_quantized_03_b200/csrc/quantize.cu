@@ -55,30 +55,30 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     block_max_store(m, partials + blockIdx.x);
 }
 
-// amax of the random Hadamard transform along the rows: each work item is 16 rows x 8
-// columns (16 coalesced 16-byte loads), i.e. eight 16-element transforms.
+// amax of the random Hadamard transform along the rows: each work item is 16 rows x 4 columns
+// (16 coalesced 8-byte loads), i.e. four 16-element transforms.
 __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x,
                                                        int64_t rows, int64_t cols, int64_t ld,
                                                        uint32_t sign_mask,
                                                        uint32_t* __restrict__ partials)
 {
-    const int64_t cpr = cols >> 3;
+    const int64_t cpr = cols >> 2;  // 8-byte column groups per row
     const int64_t total = (rows >> 4) * cpr;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     uint32_t m = 0;
     for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
          i += stride) {
         const int64_t g = i / cpr, c = i - g * cpr;
-        const uint16_t* base = x + (g << 4) * ld + (c << 3);
-        uint4 v[16];
+        const uint16_t* base = x + (g << 4) * ld + (c << 2);
+        uint2 v[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = __ldg(reinterpret_cast<const uint4*>(base + k * ld));
+        for (int k = 0; k < 16; ++k) v[k] = __ldg(reinterpret_cast<const uint2*>(base + k * ld));
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 4; ++j) {
             float y[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const uint32_t w = j < 2 ? v[k].x : j < 4 ? v[k].y : j < 6 ? v[k].z : v[k].w;
+                const uint32_t w = j < 2 ? v[k].x : v[k].y;
                 y[k] = (j & 1) ? bf16_hi(w) : bf16_lo(w);
             }
             rht16(y, sign_mask);
@@ -139,68 +139,106 @@ __device__ __forceinline__ void zero_scale_padding(uint8_t* scales, int64_t rows
 
 // ------------------------------------------------------------------------------------------
 // Pass 2a: row-wise 1x16 quantization (x quantized along its columns).
-// Lane l of a warp owns 16-byte chunk (base + l): 8 elements; the two lanes of a 16-element
-// block exchange their maxima with one shuffle; lane 8k gathers the 4 scales of its
-// 64-element group into one 32-bit word.  With SR the Philox counter of the chunk is its
-// flat index (element index / 8).
+// A warp takes 128 consecutive 16-byte chunks (8 elements each) per iteration: lane l owns
+// chunks base + l + 32 u, u = 0..3, so each of the four loads, issued together, is one
+// coalesced 512-byte access.  The two lanes of a 16-element block exchange their maxima with
+// one shuffle; lane 8k gathers the 4 scales of its 64-element group into one 32-bit word.
+// With SR the Philox counter of a chunk is its flat index (element index / 8).
 // ------------------------------------------------------------------------------------------
+template <bool SR>
+__device__ __forceinline__ uint32_t encode8(const float* e, const BlockScale& bs, const Philox& ph,
+                                            uint64_t f, uint64_t offset)
+{
+    uint32_t packed = 0;
+    if (SR) {
+        const uint4 rnd = ph.group(f, offset);
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const float q0 = e2m1_sr_value(__fmul_rn(e[j], bs.r), lane16(rnd, j));
+            const float q1 = e2m1_sr_value(__fmul_rn(e[j + 1], bs.r), lane16(rnd, j + 1));
+            packed |= e2m1x2_rn(q0, q1) << (4 * j);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; j += 2)
+            packed |= e2m1x2_rn(__fmul_rn(e[j], bs.r), __fmul_rn(e[j + 1], bs.r)) << (4 * j);
+    }
+    return packed;
+}
+
 template <bool SR>
 __global__ void __launch_bounds__(256) quant_rowwise_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, QuantSource src,
     float* amax_out0, float* amax_out1, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, uint64_t seed, uint64_t offset, int* dev_status)
 {
+    constexpr int U = 4;
     const TensorScale ts = fold_amax(src, amax_out0, amax_out1, dev_status);
     const Philox philox(seed);
     const int lane = threadIdx.x & 31;
     const int64_t cpr = cols >> 3;
     const int64_t gpr = cols >> 6;
     const int64_t total = rows * cpr;                   // chunks (multiple of 8)
-    const int64_t nwork = (total + 31) >> 5;            // warp-sized pieces
+    const int64_t nwork = (total + 32 * U - 1) / (32 * U);
     const int64_t wstride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int64_t wfirst = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const bool contiguous = ld == cols;
 
-    for (int64_t w = wfirst; w < nwork; w += wstride) {
-        const int64_t f = ((nwork - 1 - w) << 5) + lane;  // reverse order (L2 reuse)
-        const bool valid = f < total;
-        int64_t r = 0, c8 = 0;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (valid) {
-            r = f / cpr;
-            c8 = f - r * cpr;
-            v = __ldg(reinterpret_cast<const uint4*>(x + r * ld) + c8);
-        }
-        float e[8];
-        unpack8(v, e);
-        float m = 0.0f;
+    // Row and column of this lane's first chunk, kept up to date without dividing: each
+    // iteration moves back by D = wstride * 128 chunks = dq rows and dr chunks.
+    const int64_t D = wstride * (32 * U);
+    const int64_t dq = D / cpr, dr = D - dq * cpr;
+    int64_t f0 = (nwork - 1 - wfirst) * (32 * U) + lane;
+    int64_t r = f0 / cpr, c8 = f0 - r * cpr;
+    for (int64_t w = wfirst; w < nwork; w += wstride, f0 -= D) {
+        int64_t rr[U], cc[U];
+        uint4 v[U];
+        {
+            int64_t ru = r, cu = c8;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(e[j]));
-        const float b = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-        const BlockScale bs = block_scale(b, ts.s_enc);
-        uint32_t packed = 0;
-        if (SR) {
-            const uint4 rnd = philox.group(static_cast<uint64_t>(f), offset);
-#pragma unroll
-            for (int j = 0; j < 8; j += 2) {
-                const float q0 = e2m1_sr_value(__fmul_rn(e[j], bs.r), lane16(rnd, j));
-                const float q1 = e2m1_sr_value(__fmul_rn(e[j + 1], bs.r), lane16(rnd, j + 1));
-                packed |= e2m1x2_rn(q0, q1) << (4 * j);
+            for (int u = 0; u < U; ++u) {
+                rr[u] = ru;
+                cc[u] = cu;
+                const int64_t f = f0 + 32 * u;
+                v[u] = make_uint4(0, 0, 0, 0);
+                if (f < total)
+                    v[u] = __ldg(contiguous ? reinterpret_cast<const uint4*>(x) + f
+                                            : reinterpret_cast<const uint4*>(x + ru * ld) + cu);
+                cu += 32;
+                while (cu >= cpr) {
+                    cu -= cpr;
+                    ++ru;
+                }
             }
-        } else {
-#pragma unroll
-            for (int j = 0; j < 8; j += 2)
-                packed |= e2m1x2_rn(__fmul_rn(e[j], bs.r), __fmul_rn(e[j + 1], bs.r)) << (4 * j);
         }
-        const uint32_t sf = ts.nonfinite ? 0u : bs.sf;
-        if (ts.nonfinite) packed = 0;
-        const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sf, 2);
-        const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sf, 4);
-        const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sf, 6);
-        if (valid) {
-            reinterpret_cast<uint32_t*>(codes)[f] = packed;
-            if ((lane & 7) == 0)
-                *reinterpret_cast<uint32_t*>(scales + sf_offset(r, c8 >> 1, gpr)) =
-                    sf | (s1 << 8) | (s2 << 16) | (s3 << 24);
+        r -= dq;
+        c8 -= dr;
+        if (c8 < 0) {
+            c8 += cpr;
+            --r;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t f = f0 + 32 * u;
+            float e[8];
+            unpack8(v[u], e);
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(e[j]));
+            const float b = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            const BlockScale bs = block_scale(b, ts.s_enc);
+            uint32_t packed = encode8<SR>(e, bs, philox, static_cast<uint64_t>(f), offset);
+            const uint32_t sf = ts.nonfinite ? 0u : bs.sf;
+            if (ts.nonfinite) packed = 0;
+            const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sf, 2);
+            const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sf, 4);
+            const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sf, 6);
+            if (f < total) {
+                reinterpret_cast<uint32_t*>(codes)[f] = packed;
+                if ((lane & 7) == 0)
+                    *reinterpret_cast<uint32_t*>(scales + sf_offset(rr[u], cc[u] >> 1, gpr)) =
+                        sf | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            }
         }
     }
     zero_scale_padding(scales, rows, cols,
@@ -381,7 +419,7 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
 
 int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count)
 {
-    const int64_t items = rht ? (rows / 16) * (cols / 8) : rows * (cols / 8);
+    const int64_t items = rht ? (rows / 16) * (cols / 4) : rows * (cols / 8);
     const int64_t per_cta = rht ? 256 : 256 * 4;
     int64_t g = (items + per_cta - 1) / per_cta;
     const int64_t cap = static_cast<int64_t>(sm_count) * 8;
@@ -406,7 +444,7 @@ cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, 
                                  uint8_t* codes, uint8_t* scales, bool sr, uint64_t seed,
                                  uint64_t offset, int* dev_status, int sm_count, cudaStream_t s)
 {
-    const int64_t warps = (rows * (cols >> 3) + 31) / 32;
+    const int64_t warps = (rows * (cols >> 3) + 127) / 128;
     int64_t grid = (warps + 7) / 8;
     const int64_t cap = static_cast<int64_t>(sm_count) * 16;
     if (grid > cap) grid = cap;
