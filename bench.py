@@ -506,6 +506,84 @@ def run_kernel_case(args):
     return 0
 
 
+SWEEP_MODES = {
+    # name: (flags, rht, outputs)
+    "1x16_rtn_row": (1, False, 1),
+    "1x16_rtn_col": (2, False, 1),
+    "1x16_rtn_rowcol": (3, False, 2),
+    "16x16_2d_rowcol": (1 | 2 | 4, False, 2),
+    "1x16_sr_row": (1 | 8, False, 1),
+    "1x16_sr_col": (2 | 8, False, 1),
+    "rht_1x16_sr_col": (8, True, 1),
+    "rht_1x16_rtn_col": (0, True, 1),
+}
+
+
+def run_sweep(args):
+    """Quantizer bandwidth sweep: bf16 tensors of 2^n elements in rows of 4096 (N(0,1) with 1 %
+    x50 outliers), each mode timed over `steps` calls after `warmup`; one JSON line per point.
+    GB/s counts the algorithmic bytes of a call: two 2-byte reads of every element (the amax
+    pass and the quantize pass) plus 0.5625 bytes of codes and scales per element per output."""
+    import torch
+    from nvfp4_bit_quantized_03_b200 import binding as B
+    peaks = _peaks()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    lo, hi = args.sweep_min, args.sweep_max
+    for log2n in range(lo, hi + 1):
+        rows, cols = synth.quant_sweep_shape(log2n)
+        ws = torch.empty((max(B.workspace_bytes(rows, cols, 1 | 2 | 8), 16),), dtype=torch.uint8,
+                         device=dev)
+        x = torch.from_numpy(synth.activations((rows, cols), seed=synth.QUANT_SWEEP_SEED)
+                             .view(np.int16)).view(torch.bfloat16).to(dev)
+        n = rows * cols
+        for name, (flags, rht, outs) in SWEEP_MODES.items():
+            qr = B.QuantizedTensor(rows, cols, dev) if flags & 1 else None
+            qc = B.QuantizedTensor(cols, rows, dev) if (flags & 2 or rht) else None
+            if rht:
+                fn = lambda: B.rht_quantize(x, 0x5A3C, flags, seed=1, out_col=qc, workspace=ws)  # noqa: E731
+            else:
+                fn = lambda: B.quantize(x, flags, seed=1, out_row=qr, out_col=qc, workspace=ws)  # noqa: E731
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            # the calls are replayed from a CUDA graph so that small sizes time the GPU, not
+            # the Python dispatch; a graph that cannot be captured falls back to plain calls
+            graph = None
+            try:
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    for _ in range(args.steps):
+                        fn()
+                graph = g
+            except RuntimeError:
+                torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            if graph is not None:
+                graph.replay()
+            torch.cuda.synchronize()
+            e0.record()
+            if graph is not None:
+                graph.replay()
+            else:
+                for _ in range(args.steps):
+                    fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            graph_used = graph is not None
+            del graph
+            gbs = n * (4 + outs * (0.5 + 1 / 16)) / (ms / 1e3) / 1e9
+            print(json.dumps({"sweep": "quantize", "log2n": log2n, "mode": name, "ms": ms,
+                              "graph": graph_used,
+                              "input_fits_in_l2": 2 * n < 126 * 2**20,
+                              "gbps": gbs, "frac_of_measured_hbm": gbs / peaks["hbm_gbs"]}),
+                  flush=True)
+            del qr, qc
+        del x
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -516,12 +594,18 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", choices=["gemm", "rowwise", "tile2d", "rht"], default=None,
                     help="time one kernel family alone at the workload's shapes (profiling)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="quantizer bandwidth sweep over 2^n-element tensors (one line per point)")
+    ap.add_argument("--sweep-min", type=int, default=20)
+    ap.add_argument("--sweep-max", type=int, default=30)
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
         return run_reference(args)
     if args.kernel:
         return run_kernel_case(args)
+    if args.sweep:
+        return run_sweep(args)
     return run_ours(args)
 
 

@@ -76,12 +76,6 @@ struct Philox {
     }
 };
 
-__device__ __forceinline__ uint32_t lane16(const uint4& w, int j)
-{
-    const uint32_t word = (j >> 1) == 0 ? w.x : (j >> 1) == 1 ? w.y : (j >> 1) == 2 ? w.z : w.w;
-    return (j & 1) ? (word >> 16) : (word & 0xFFFFu);
-}
-
 // ---- scales ----------------------------------------------------------------------------
 
 // Tensor encode scale: 2688 / amax (6 * 448 / amax); 1 for amax == 0; FLT_MAX on overflow.
@@ -141,24 +135,103 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi)
     return r & 0xFFu;
 }
 
-// Stochastic rounding of v to the E2M1 grid with the 16-bit random integer r16: the
-// magnitude goes up to the next grid point iff r16 < p * 65536, p the position of |v|
-// between its grid neighbours.  The grid spacing is 0.5 below 2, 1 below 4 and 2 from 4 on,
-// so t = |v| / spacing is exact and p = frac(t).  For integers, r16 < p * 65536 holds iff
-// r16 < ceil(p * 65536) = ceil(t * 65536) - floor(t) * 65536; with xi = ceil(t * 65536) (an
-// exact conversion, t * 65536 being an exact FP32 product) the rounded grid index is
-// (xi >> 16) + (r16 < (xi & 0xFFFF)) -- when the fraction rounds up to a whole 65536 the carry
-// is already in xi >> 16 and the comparison is false.  The result index * spacing is a grid
-// point (anything from 6 up saturates to 6 in the conversion) and keeps the sign of v.
-__device__ __forceinline__ float e2m1_sr_value(float v, uint32_t r16)
+// ---- stochastic rounding to E2M1 ---------------------------------------------------------
+// The reading: the magnitude goes up to the next grid point iff r16 < p * 65536, p the
+// position of |v| between its grid neighbours, r16 a 16-bit random integer; from 6 up it is 6.
+//
+// mu(a) = min(2a, a + 2, a/2 + 4, 7) maps the grid magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6}
+// onto the codes 0..7 and is linear between neighbours, so mu(a) = i + p with i the code of
+// the lower neighbour.  Then i + [r16 < 65536 p] = ceil(mu(a) - r16 / 65536): for an integer
+// r16, r16 < 65536 p holds iff p - r16 / 65536 > 0.  The kernel evaluates it exactly on the
+// 65536-scaled values m = 65536 mu(a):
+//   * the lines a * 2^17 (exact), a * 2^16 + 2^17 and a * 2^15 + 2^18 rounded upward, and the
+//     constant 7 * 2^16: their minimum m' lies in [m, RU(m)];
+//   * P = RU(m' + 2^23) = 2^23 + ceil(m) (the spacing of FP32 at 2^23 is 1, and every
+//     integer from m up to ceil(m) is representable, so rounding m up first changes nothing);
+//   * Q = P - (2^23 + r16) = ceil(m) - r16, exact (integers below 2^24);
+//   * k = RU(Q / 2^16 + 1.5 * 2^23) = 1.5 * 2^23 + ceil(Q / 2^16) = 1.5 * 2^23 + code
+//     (ceil(ceil(m) - r16) / 2^16) = ceil((m - r16) / 2^16) for integer r16, and Q / 2^16 lies
+//     in (-1, 7], where FP32 spacing is 1 around 1.5 * 2^23).
+// The low byte of k's bit pattern is the magnitude code.  Every operation is an FP32 FMA-pipe
+// instruction with a fixed rounding direction, so the result does not depend on contraction.
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
-    const float a = fabsf(v);
-    const float c = a < 2.0f ? 131072.0f : (a < 4.0f ? 65536.0f : 32768.0f);  // 65536 / spacing
-    const float step = a < 2.0f ? 0.5f : (a < 4.0f ? 1.0f : 2.0f);
-    uint32_t xi;
-    asm("cvt.rpi.sat.u32.f32 %0, %1;" : "=r"(xi) : "f"(__fmul_rn(a, c)));
-    const uint32_t idx = (xi >> 16) + (r16 < (xi & 0xFFFFu) ? 1u : 0u);
-    return copysignf(__fmul_rn(__uint2float_rn(idx), step), v);
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+__device__ __forceinline__ float min3f(float a, float b, float c)
+{
+    float d;
+    asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Bit pattern of the FP32 value 2^23 + r16 for half h (0: low, 1: high) of a 32-bit random
+// word: the two bytes of the half under the exponent byte 0x4B.
+__device__ __forceinline__ uint32_t rand16_as_f32_bits(uint32_t word, int h)
+{
+    return prmt(word, 0x4B000000u, h ? 0x7632u : 0x7610u);
+}
+
+// Magnitude code of a >= 0 stochastically rounded with the random value whose FP32 pattern is
+// rbits = bits(2^23 + r16); the code is the low byte of the returned pattern.
+__device__ __forceinline__ uint32_t e2m1_sr_code(float a, uint32_t rbits)
+{
+    const float l0 = __fmul_rn(a, 131072.0f);
+    const float l1 = __fmaf_ru(a, 65536.0f, 131072.0f);
+    const float l2 = __fmaf_ru(a, 32768.0f, 262144.0f);
+    const float m = fminf(min3f(l0, l1, l2), 458752.0f);
+    const float P = __fadd_ru(m, 8388608.0f);
+    const float Q = __fsub_rn(P, __uint_as_float(rbits));
+    return __float_as_uint(__fmaf_ru(Q, 0x1p-16f, 12582912.0f));
+}
+
+// Eight codes held in the low bytes of k[0..7] packed as nibbles, element j at bits 4j..4j+3.
+__device__ __forceinline__ uint32_t pack8_low_bytes(const uint32_t* k)
+{
+    const uint32_t even = prmt(prmt(k[0], k[2], 0x0040u), prmt(k[4], k[6], 0x0040u), 0x5410u);
+    const uint32_t odd = prmt(prmt(k[1], k[3], 0x0040u), prmt(k[5], k[7], 0x0040u), 0x5410u);
+    return even | (odd << 4);
+}
+
+// E2M1 sign bits (bit 4j + 3) of the 8 bf16 values of a 16-byte vector.  A prmt selector
+// nibble with its top bit set fills the result byte with the top bit of the selected byte;
+// the sign of value 2i is the top bit of byte 1 of word i, that of value 2i + 1 of byte 3.
+__device__ __forceinline__ uint32_t signs8_bf16(const uint4& v)
+{
+    const uint32_t lo4 = prmt(v.x, v.y, 0xFDB9u);  // byte i: 0xFF iff value i < 0
+    const uint32_t hi4 = prmt(v.z, v.w, 0xFDB9u);  // byte i: 0xFF iff value 4 + i < 0
+    const uint32_t even = prmt(lo4, hi4, 0x6420u);
+    const uint32_t odd = prmt(lo4, hi4, 0x7531u);
+    return (even & 0x08080808u) | (odd & 0x80808080u);
+}
+
+// E2M1 sign bits (bit 4j + 3) of 8 FP32 values (the top bit of byte 3 of each).
+__device__ __forceinline__ uint32_t signs8_f32(const float* y)
+{
+    const uint32_t even = prmt(prmt(__float_as_uint(y[0]), __float_as_uint(y[2]), 0x00FBu),
+                               prmt(__float_as_uint(y[4]), __float_as_uint(y[6]), 0x00FBu),
+                               0x5410u);
+    const uint32_t odd = prmt(prmt(__float_as_uint(y[1]), __float_as_uint(y[3]), 0x00FBu),
+                              prmt(__float_as_uint(y[5]), __float_as_uint(y[7]), 0x00FBu),
+                              0x5410u);
+    return (even & 0x08080808u) | (odd & 0x80808080u);
+}
+
+// Eight stochastically rounded E2M1 codes of the values x[0..7] scaled by r, with the random
+// word group rnd (value j takes half j & 1 of word j >> 1) and the sign bits `signs`.
+__device__ __forceinline__ uint32_t e2m1x8_sr(const float* x, float r, const uint4& rnd,
+                                             uint32_t signs)
+{
+    uint32_t k[8];
+    const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        k[j] = e2m1_sr_code(__fmul_rn(fabsf(x[j]), r), rand16_as_f32_bits(w[j >> 1], j & 1));
+    return pack8_low_bytes(k) | signs;
 }
 
 // ---- random Hadamard transform ----------------------------------------------------------

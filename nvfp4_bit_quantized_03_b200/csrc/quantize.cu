@@ -146,23 +146,14 @@ __device__ __forceinline__ void zero_scale_padding(uint8_t* scales, int64_t rows
 // With SR the Philox counter of a chunk is its flat index (element index / 8).
 // ------------------------------------------------------------------------------------------
 template <bool SR>
-__device__ __forceinline__ uint32_t encode8(const float* e, const BlockScale& bs, const Philox& ph,
-                                            uint64_t f, uint64_t offset)
+__device__ __forceinline__ uint32_t encode8(const uint4& v, const float* e, const BlockScale& bs,
+                                            const Philox& ph, uint64_t f, uint64_t offset)
 {
+    if (SR) return e2m1x8_sr(e, bs.r, ph.group(f, offset), signs8_bf16(v));
     uint32_t packed = 0;
-    if (SR) {
-        const uint4 rnd = ph.group(f, offset);
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-            const float q0 = e2m1_sr_value(__fmul_rn(e[j], bs.r), lane16(rnd, j));
-            const float q1 = e2m1_sr_value(__fmul_rn(e[j + 1], bs.r), lane16(rnd, j + 1));
-            packed |= e2m1x2_rn(q0, q1) << (4 * j);
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 8; j += 2)
-            packed |= e2m1x2_rn(__fmul_rn(e[j], bs.r), __fmul_rn(e[j + 1], bs.r)) << (4 * j);
-    }
+    for (int j = 0; j < 8; j += 2)
+        packed |= e2m1x2_rn(__fmul_rn(e[j], bs.r), __fmul_rn(e[j + 1], bs.r)) << (4 * j);
     return packed;
 }
 
@@ -227,7 +218,7 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(
             for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(e[j]));
             const float b = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             const BlockScale bs = block_scale(b, ts.s_enc);
-            uint32_t packed = encode8<SR>(e, bs, philox, static_cast<uint64_t>(f), offset);
+            uint32_t packed = encode8<SR>(v[u], e, bs, philox, static_cast<uint64_t>(f), offset);
             const uint32_t sf = ts.nonfinite ? 0u : bs.sf;
             if (ts.nonfinite) packed = 0;
             const uint32_t s1 = __shfl_down_sync(0xFFFFFFFFu, sf, 2);
@@ -267,16 +258,14 @@ __device__ __forceinline__ void encode16(const float* y, const BlockScale& bs, c
     uint32_t p[2] = {0u, 0u};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        uint4 rnd = make_uint4(0, 0, 0, 0);
-        if (SR) rnd = ph.group((e0 >> 3) + h, offset);
+        if (SR) {
+            p[h] = e2m1x8_sr(y + 8 * h, bs.r, ph.group((e0 >> 3) + h, offset),
+                             signs8_f32(y + 8 * h));
+        } else {
 #pragma unroll
-        for (int j = 0; j < 8; j += 2) {
-            float a = __fmul_rn(y[8 * h + j], bs.r), b = __fmul_rn(y[8 * h + j + 1], bs.r);
-            if (SR) {
-                a = e2m1_sr_value(a, lane16(rnd, j));
-                b = e2m1_sr_value(b, lane16(rnd, j + 1));
-            }
-            p[h] |= e2m1x2_rn(a, b) << (4 * j);
+            for (int j = 0; j < 8; j += 2)
+                p[h] |= e2m1x2_rn(__fmul_rn(y[8 * h + j], bs.r), __fmul_rn(y[8 * h + j + 1], bs.r))
+                        << (4 * j);
         }
     }
     w0 = p[0];
