@@ -192,18 +192,18 @@ class Step:
         return sum(3 * f for f in self.flops_per_gemm)
 
     def quant_bytes(self):
-        """Algorithmic quantizer bytes of one step: per operand, the amax read (2 B/elem),
-        the quantize read (2 B/elem) and the codes + scales write (0.5 + 1/16 B/elem)."""
+        """Algorithmic quantizer bytes of one step: each of X, W and dY is read twice (the amax
+        pass and the quantize pass, 2 B/elem each) and written in its two GEMM orientations
+        (0.5 + 1/16 B/elem each): 5.125 B/elem."""
         total = 0
         for L in self.layers:
             lin = L["lin"]
-            for n in (lin.T * lin.I, lin.O * lin.I, lin.T * lin.O, lin.O * lin.I,
-                      lin.T * lin.O, lin.T * lin.I):
-                total += n * (2 + 2 + 0.5 + 1 / 16)
+            for n in (lin.T * lin.I, lin.O * lin.I, lin.T * lin.O):
+                total += n * (2 + 2 + 2 * (0.5 + 1 / 16))
         return total
 
     def n_quant_launches(self):
-        return 2 * 2 * 3 * len(self.layers)   # (amax + quantize) x 2 operands x 3 GEMMs
+        return 2 * 3 * len(self.layers)   # (amax + quantize) x (X, W, dY)
 
     def n_gemm_launches(self):
         return 3 * len(self.layers)
@@ -227,24 +227,23 @@ class Step:
 
         for L in self.layers:
             X, W, dY, out = L["X"], L["W"], L["dY"], L["out"]
-            a, b = L["fprop"]
-            timed("quant", lambda: B.quantize(W, B.ROWWISE | B.BLOCK2D, out_row=b, workspace=ws,
-                                              dev_status=st))
-            timed("quant", lambda: B.quantize(X, B.ROWWISE, out_row=a, workspace=ws,
-                                              dev_status=st))
-            timed("gemm", lambda: B.gemm(a, b, out=out["fprop"], dev_status=st))
-            a, b = L["dgrad"]
-            timed("quant", lambda: B.quantize(W, B.COLWISE | B.BLOCK2D, out_col=b, workspace=ws,
-                                              dev_status=st))
-            timed("quant", lambda: B.quantize(dY, B.ROWWISE | B.SR, seed=self.seed, offset=0,
-                                              out_row=a, workspace=ws, dev_status=st))
-            timed("gemm", lambda: B.gemm(a, b, out=out["dgrad"], dev_status=st))
-            a, b = L["wgrad"]
-            timed("quant", lambda: B.rht_quantize(dY, self.mask, B.SR, seed=self.seed, offset=1,
-                                                  out_col=a, workspace=ws, dev_status=st))
-            timed("quant", lambda: B.rht_quantize(X, self.mask, 0, out_col=b, workspace=ws,
-                                                  dev_status=st))
-            timed("gemm", lambda: B.gemm(a, b, out=out["wgrad"], dev_status=st))
+            # Each operand is quantized once into both orientations its two GEMMs read:
+            # W with 16x16 scales (row-wise for fprop, column-wise for dgrad); X row-wise
+            # (fprop) and RHT'd column-wise (wgrad); dY row-wise with SR stream 0 (dgrad) and
+            # RHT'd column-wise with SR stream 1 (wgrad).
+            xa, wb = L["fprop"]
+            dya, wcb = L["dgrad"]
+            dyc, xcb = L["wgrad"]
+            timed("quant", lambda: B.quantize(W, B.ROWWISE | B.COLWISE | B.BLOCK2D, out_row=wb,
+                                              out_col=wcb, workspace=ws, dev_status=st))
+            timed("quant", lambda: B.quantize_row_rht(X, self.mask, 0, out_row=xa, out_col=xcb,
+                                                      workspace=ws, dev_status=st))
+            timed("quant", lambda: B.quantize_row_rht(dY, self.mask, B.SR, seed=self.seed,
+                                                      offset=0, out_row=dya, out_col=dyc,
+                                                      workspace=ws, dev_status=st))
+            timed("gemm", lambda: B.gemm(xa, wb, out=out["fprop"], dev_status=st))
+            timed("gemm", lambda: B.gemm(dya, wcb, out=out["dgrad"], dev_status=st))
+            timed("gemm", lambda: B.gemm(dyc, xcb, out=out["wgrad"], dev_status=st))
 
     def upload(self):
         """Host -> device copies of this step's inputs (from pinned memory)."""
@@ -432,7 +431,7 @@ def run_ours(args):
             "config": {"workload": wl.name, "tokens": 8192, "d_model": 5120, "d_ff": 20480,
                        "gemms_per_step": 6, "gemm_tflop_per_step": step.gemm_flops / 1e12,
                        "outputs": "Y and dX bf16, dW fp32",
-                       "recipe": "W 16x16 RTN, X 1x16 RTN, dY 1x16 SR, wgrad RHT16 (+SR on dY)",
+                       "recipe": "W 16x16 RTN (row+col, one pass), X 1x16 RTN + RHT16 col (one pass), dY 1x16 SR + RHT16 SR col (one pass)",
                        "l2": "inputs larger than L2: 1.26 GB of bf16 inputs read per step",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
@@ -484,10 +483,16 @@ def run_kernel_case(args):
         elif args.kernel == "tile2d":
             q = B.QuantizedTensor(F, T, dev)
             fn = lambda: B.quantize(x, B.COLWISE | B.BLOCK2D, out_col=q, workspace=ws)  # noqa: E731
-        else:
+        elif args.kernel == "rht":
             q = B.QuantizedTensor(F, T, dev)
             fn = lambda: B.rht_quantize(x, 0x5A3C, B.SR, seed=1, out_col=q, workspace=ws)  # noqa: E731
-        work, unit, peak = n * (4 + 0.5 + 1 / 16) / 1e9, "GB/s", peaks["hbm_gbs"]
+        else:
+            q = B.QuantizedTensor(T, F, dev)
+            q2 = B.QuantizedTensor(F, T, dev)
+            fn = lambda: B.quantize_row_rht(x, 0x5A3C, B.SR, seed=1, out_row=q, out_col=q2,  # noqa: E731
+                                            workspace=ws)
+        outs = 2 if args.kernel == "dual" else 1
+        work, unit, peak = n * (4 + outs * (0.5 + 1 / 16)) / 1e9, "GB/s", peaks["hbm_gbs"]
         shape = f"{T} x {F} bf16, amax pass + quantize pass"
     for _ in range(args.warmup):
         fn()
@@ -516,6 +521,8 @@ SWEEP_MODES = {
     "1x16_sr_col": (2 | 8, False, 1),
     "rht_1x16_sr_col": (8, True, 1),
     "rht_1x16_rtn_col": (0, True, 1),
+    "dual_rtn_row_rhtcol": (0, "dual", 2),
+    "dual_sr_row_rhtcol": (8, "dual", 2),
 }
 
 
@@ -537,9 +544,13 @@ def run_sweep(args):
                              .view(np.int16)).view(torch.bfloat16).to(dev)
         n = rows * cols
         for name, (flags, rht, outs) in SWEEP_MODES.items():
-            qr = B.QuantizedTensor(rows, cols, dev) if flags & 1 else None
+            dual = rht == "dual"
+            qr = B.QuantizedTensor(rows, cols, dev) if (flags & 1 or dual) else None
             qc = B.QuantizedTensor(cols, rows, dev) if (flags & 2 or rht) else None
-            if rht:
+            if dual:
+                fn = lambda: B.quantize_row_rht(x, 0x5A3C, flags, seed=1, out_row=qr,  # noqa: E731
+                                                out_col=qc, workspace=ws)
+            elif rht:
                 fn = lambda: B.rht_quantize(x, 0x5A3C, flags, seed=1, out_col=qc, workspace=ws)  # noqa: E731
             else:
                 fn = lambda: B.quantize(x, flags, seed=1, out_row=qr, out_col=qc, workspace=ws)  # noqa: E731
@@ -592,7 +603,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["gemm", "rowwise", "tile2d", "rht"], default=None,
+    ap.add_argument("--kernel", choices=["gemm", "rowwise", "tile2d", "rht", "dual"], default=None,
                     help="time one kernel family alone at the workload's shapes (profiling)")
     ap.add_argument("--sweep", action="store_true",
                     help="quantizer bandwidth sweep over 2^n-element tensors (one line per point)")

@@ -123,8 +123,9 @@ const char* nvfp4_status_string(nvfp4_status status);
 size_t nvfp4_codes_bytes(int64_t rows, int64_t cols);
 size_t nvfp4_scales_bytes(int64_t rows, int64_t cols);
 
-/* Device workspace needed by nvfp4_quantize / nvfp4_rht_quantize for a rows x cols input
- * (the per-block partial maxima of the amax pass).  0 with NVFP4_AMAX_GIVEN. */
+/* Device workspace needed by nvfp4_quantize / nvfp4_rht_quantize / nvfp4_quantize_row_rht
+ * for a rows x cols input (the per-block partial maxima of the amax pass).  0 with
+ * NVFP4_AMAX_GIVEN. */
 size_t nvfp4_workspace_bytes(int64_t rows, int64_t cols, unsigned flags);
 
 /* Device workspace needed by each nvfp4_linear_* call for T tokens, I in-features and O
@@ -177,6 +178,29 @@ nvfp4_status nvfp4_rht_quantize(const void* x_bf16, int64_t rows, int64_t cols, 
                                 uint16_t sign_mask, unsigned flags, uint64_t seed,
                                 uint64_t offset, const nvfp4_operand* out_col,
                                 void* workspace, int* dev_status, void* stream);
+
+/*
+ * Both quantizations a linear layer needs of one activation or output gradient x (T x C:
+ * tokens x features), from one amax pass and one quantize pass over x.  [P1 Formato NVFP4;
+ * RHT; Escalado 2D y Redondeo Estocastico]: x feeds the forward (or data-gradient) GEMM
+ * quantized along its features, and the weight-gradient GEMM random-Hadamard-transformed and
+ * quantized along its tokens.
+ *   out_row  : rows x cols operand, exactly what nvfp4_quantize(x, NVFP4_ROWWISE | (flags &
+ *              NVFP4_SR), seed, offset) writes (amax = max |x|).
+ *   out_col  : cols x rows operand, exactly what nvfp4_rht_quantize(x, sign_mask, flags, seed,
+ *              offset + 1) writes (amax = max |RHT(x)|): the two SR streams are offset and
+ *              offset + 1, as for the data- and weight-gradient operands of one dY.
+ *   flags    : NVFP4_SR and/or NVFP4_AMAX_GIVEN (both amaxes are then read from out_row->amax
+ *              and out_col->amax); other bits are rejected with NVFP4_ERR_ARG.
+ *   workspace: nvfp4_workspace_bytes(rows, cols, flags) device bytes (NULL if 0).
+ * Shape rules: rows and cols multiples of 64, ld >= cols, ld % 8 == 0.  Each output is
+ * zero-filled on its own when its amax is not finite (NVFP4_DEVSTAT_NONFINITE is set).
+ */
+nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                    uint16_t sign_mask, unsigned flags, uint64_t seed,
+                                    uint64_t offset, const nvfp4_operand* out_row,
+                                    const nvfp4_operand* out_col, void* workspace,
+                                    int* dev_status, void* stream);
 
 /*
  * Block-scaled FP4 GEMM on the tcgen05 tensor cores: D = A . B^T.

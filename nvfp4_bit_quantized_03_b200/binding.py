@@ -63,6 +63,9 @@ def lib():
         L.nvfp4_rht_quantize.argtypes = [vp, i64, i64, i64, u16, ctypes.c_uint, u64, u64, op, vp,
                                          vp, vp]
         L.nvfp4_rht_quantize.restype = i32
+        L.nvfp4_quantize_row_rht.argtypes = [vp, i64, i64, i64, u16, ctypes.c_uint, u64, u64, op,
+                                             op, vp, vp, vp]
+        L.nvfp4_quantize_row_rht.restype = i32
         L.nvfp4_gemm.argtypes = [op, op, vp, i32, i64, vp, vp]
         L.nvfp4_gemm.restype = i32
         L.nvfp4_linear_fprop.argtypes = [vp, vp, i64, i64, i64, vp, i32, vp, vp, vp]
@@ -196,6 +199,26 @@ def rht_quantize(x, sign_mask, flags=0, seed=0, offset=0, out_col=None, workspac
                                   _stream(stream))
     _check(st, "nvfp4_rht_quantize")
     return out_col
+
+
+def quantize_row_rht(x, sign_mask, flags=0, seed=0, offset=0, out_row=None, out_col=None,
+                     workspace=None, dev_status=None, stream=None):
+    """nvfp4_quantize_row_rht: x row-wise (stream `offset`) and x^T RHT'd column-wise (stream
+    `offset + 1`) from one amax pass and one quantize pass."""
+    assert x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1
+    rows, cols = x.shape
+    if out_row is None:
+        out_row = QuantizedTensor(rows, cols, x.device)
+    if out_col is None:
+        out_col = QuantizedTensor(cols, rows, x.device)
+    if workspace is None:
+        workspace = _workspace(workspace_bytes(rows, cols, flags), x.device)
+    op_r, op_c = out_row.operand(), out_col.operand()
+    st = lib().nvfp4_quantize_row_rht(_ptr(x), rows, cols, x.stride(0), sign_mask, flags, seed,
+                                      offset, ctypes.byref(op_r), ctypes.byref(op_c),
+                                      _ptr(workspace), _ptr(dev_status), _stream(stream))
+    _check(st, "nvfp4_quantize_row_rht")
+    return out_row, out_col
 
 
 def _check_out(out, rows, cols, what):

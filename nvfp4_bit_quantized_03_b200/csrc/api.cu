@@ -117,6 +117,26 @@ uint32_t philox_word0(uint64_t seed, uint32_t c0, uint32_t c1, uint32_t c2, uint
     return c0;
 }
 
+// Shape, alignment and pointer checks shared by the quantizer entry points.
+nvfp4_status check_input(const void* x, int64_t rows, int64_t cols, int64_t ld, bool want_row,
+                         bool want_col, const nvfp4_operand* out_row,
+                         const nvfp4_operand* out_col, bool given, const void* workspace)
+{
+    if (!x) return NVFP4_ERR_NULL;
+    if (rows < 16 || cols < 16 || rows >= kMaxDim || cols >= kMaxDim || rows % 16 || cols % 16 ||
+        ld < cols)
+        return NVFP4_ERR_SHAPE;
+    if (want_row && cols % 64) return NVFP4_ERR_SHAPE;
+    if (want_col && rows % 64) return NVFP4_ERR_SHAPE;
+    if (ld % 8 || !aligned16(x)) return NVFP4_ERR_ALIGN;
+    nvfp4_status st;
+    if (want_row && (st = check_operand(out_row, rows, cols)) != NVFP4_OK) return st;
+    if (want_col && (st = check_operand(out_col, cols, rows)) != NVFP4_OK) return st;
+    if (!given && !workspace) return NVFP4_ERR_NULL;
+    if (workspace && !aligned16(workspace)) return NVFP4_ERR_ALIGN;
+    return NVFP4_OK;
+}
+
 nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld, unsigned flags,
                            bool rht, uint32_t sign_mask, uint64_t seed, uint64_t offset,
                            const nvfp4_operand* out_row, const nvfp4_operand* out_col,
@@ -131,18 +151,9 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
     if (!want_row && !want_col) return NVFP4_ERR_ARG;
     if (b2d && sr) return NVFP4_ERR_ARG;
     if (rht && (want_row || b2d)) return NVFP4_ERR_ARG;
-    if (!x) return NVFP4_ERR_NULL;
-    if (rows < 16 || cols < 16 || rows >= kMaxDim || cols >= kMaxDim || rows % 16 || cols % 16 ||
-        ld < cols)
-        return NVFP4_ERR_SHAPE;
-    if (want_row && cols % 64) return NVFP4_ERR_SHAPE;
-    if (want_col && rows % 64) return NVFP4_ERR_SHAPE;
-    if (ld % 8 || !aligned16(x)) return NVFP4_ERR_ALIGN;
-    nvfp4_status st;
-    if (want_row && (st = check_operand(out_row, rows, cols)) != NVFP4_OK) return st;
-    if (want_col && (st = check_operand(out_col, cols, rows)) != NVFP4_OK) return st;
-    if (!given && !workspace) return NVFP4_ERR_NULL;
-    if (workspace && !aligned16(workspace)) return NVFP4_ERR_ALIGN;
+    nvfp4_status st = check_input(x, rows, cols, ld, want_row, want_col, out_row, out_col,
+                                  given, workspace);
+    if (st != NVFP4_OK) return st;
     int sms = 0;
     if ((st = current_device(&sms)) != NVFP4_OK) return st;
 
@@ -180,9 +191,11 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
         a.col_scales = static_cast<uint8_t*>(out_col->scales);
         a.col_amax = out_col->amax;
     }
+    a.src_col = src;
     a.sign_mask = sign_mask;
     a.seed = seed;
     a.offset = offset;
+    a.offset_col = offset;
     a.dev_status = dev_status;
     return from_cuda(launch_quant_tile(a, want_row, want_col, b2d, rht, sr, sms, s));
 }
@@ -226,7 +239,7 @@ size_t nvfp4_workspace_bytes(int64_t rows, int64_t cols, unsigned flags)
 {
     if (rows <= 0 || cols <= 0) return 0;
     if (flags & NVFP4_AMAX_GIVEN) return 0;
-    return sizeof(uint32_t) * kMaxPartials;
+    return 2 * sizeof(uint32_t) * kMaxPartials;  // the dual mode keeps two sets of partials
 }
 
 size_t nvfp4_linear_workspace_bytes(int64_t T, int64_t I, int64_t O)
@@ -281,6 +294,59 @@ nvfp4_status nvfp4_rht_quantize(const void* x_bf16, int64_t rows, int64_t cols, 
         return NVFP4_ERR_ARG;
     return quantize_impl(x_bf16, rows, cols, ld, flags | NVFP4_COLWISE, true, sign_mask, seed,
                          offset, nullptr, out_col, workspace, dev_status, stream);
+}
+
+nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,
+                                    uint16_t sign_mask, unsigned flags, uint64_t seed,
+                                    uint64_t offset, const nvfp4_operand* out_row,
+                                    const nvfp4_operand* out_col, void* workspace,
+                                    int* dev_status, void* stream)
+{
+    if (flags & ~static_cast<unsigned>(NVFP4_SR | NVFP4_AMAX_GIVEN)) return NVFP4_ERR_ARG;
+    const bool sr = flags & NVFP4_SR, given = flags & NVFP4_AMAX_GIVEN;
+    nvfp4_status st = check_input(x_bf16, rows, cols, ld, true, true, out_row, out_col, given,
+                                  workspace);
+    if (st != NVFP4_OK) return st;
+    int sms = 0;
+    if ((st = current_device(&sms)) != NVFP4_OK) return st;
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const uint16_t* xs = static_cast<const uint16_t*>(x_bf16);
+    QuantSource src_row{}, src_col{};
+    if (given) {
+        src_row.amax_given = out_row->amax;
+        src_col.amax_given = out_col->amax;
+    } else {
+        const int grid = amax_grid(rows, cols, true, sms);
+        uint32_t* partials_rht = static_cast<uint32_t*>(workspace);
+        uint32_t* partials_plain = partials_rht + kMaxPartials;
+        src_col.partials = partials_rht;
+        src_col.n_partials = grid;
+        src_row.partials = partials_plain;
+        src_row.n_partials = grid;
+        st = from_cuda(launch_amax_dual(xs, rows, cols, ld, sign_mask, partials_rht,
+                                        partials_plain, grid, s));
+        if (st != NVFP4_OK) return st;
+    }
+    TileArgs a{};
+    a.x = xs;
+    a.rows = rows;
+    a.cols = cols;
+    a.ld = ld;
+    a.src = src_row;
+    a.src_col = src_col;
+    a.row_codes = static_cast<uint8_t*>(out_row->codes);
+    a.row_scales = static_cast<uint8_t*>(out_row->scales);
+    a.row_amax = out_row->amax;
+    a.col_codes = static_cast<uint8_t*>(out_col->codes);
+    a.col_scales = static_cast<uint8_t*>(out_col->scales);
+    a.col_amax = out_col->amax;
+    a.sign_mask = sign_mask;
+    a.seed = seed;
+    a.offset = offset;
+    a.offset_col = offset + 1;
+    a.dev_status = dev_status;
+    return from_cuda(launch_quant_tile(a, true, true, false, true, sr, sms, s));
 }
 
 nvfp4_status nvfp4_gemm(const nvfp4_operand* A, const nvfp4_operand* B, void* D, int d_dtype,

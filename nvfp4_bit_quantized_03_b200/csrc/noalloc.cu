@@ -65,7 +65,10 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows,
                                                const nvfp4_operand* out_col, int* dev_status,
                                                void* stream)
 {
-    const size_t need = nvfp4_workspace_bytes(rows, cols, flags);
+    // nvfp4_quantize keeps one set of amax partials (nvfp4_workspace_bytes also covers the
+    // dual mode's second set, which this entry point never runs).
+    const size_t need =
+        (flags & NVFP4_AMAX_GIVEN) ? 0 : sizeof(uint32_t) * static_cast<size_t>(nvfp4::kMaxPartials);
     if (need > sizeof(uint32_t) * kScratchSlots) return NVFP4_ERR_SHAPE;
     uint32_t* scratch = nullptr;
     if (need > 0) {

@@ -107,17 +107,53 @@ struct BlockScale {
     float r;      // element factor S_enc / sf (0 when sf == 0)
 };
 
-// Block scale and element factor for a block whose largest magnitude is b.
-__device__ __forceinline__ BlockScale block_scale(float b, float s_enc)
+// Correctly rounded b / 6 for a finite b >= 0, without a division instruction.
+//  * b >= 2^-125: q0 = RN(b z) with z = RN(1/6), the exact remainder r = b - 6 q0 (one FMA),
+//    and q0 + r z rounded once (one FMA) -- the correction step for a divisor known in advance
+//    (Brisebarre, Muller, Raina, "Accelerating correctly rounded floating-point division when
+//    the divisor is known in advance", IEEE Trans. Computers 53(8), 2004).
+//  * b < 2^-125: b is m 2^-149 with m its bit pattern, the quotient is m / 6 in the same units
+//    rounded to nearest even, and its bit pattern is that integer; floor(m / 6) is
+//    (m * 0xAAAAAAAB) >> 34 (Granlund, Montgomery, "Division by invariant integers using
+//    multiplication", PLDI 1994).
+// Equal to IEEE b / 6 (round to nearest even) on every finite non-negative FP32 value,
+// checked exhaustively against the FPU's division.
+__device__ __forceinline__ float div6_rn(float b)
+{
+    if (b < 0x1p-125f) {
+        const uint32_t m = __float_as_uint(b);
+        const uint32_t n = __umulhi(m, 0xAAAAAAABu) >> 2;
+        const uint32_t rem = m - 6u * n;
+        return __uint_as_float(n + ((rem > 3u || (rem == 3u && (n & 1u))) ? 1u : 0u));
+    }
+    const float z = 0x1.555556p-3f;  // RN(1/6)
+    const float q0 = __fmul_rn(b, z);
+    return __fmaf_rn(__fmaf_rn(-q0, 6.0f, b), z, q0);
+}
+
+// Element factors r = S_enc / value(sf) of all 128 E4M3 codes (FP32 division, clamped to
+// FLT_MAX; 0 for sf == 0 and for the unused NaN code 0x7F), filled by the block's first 128
+// threads.  The caller synchronizes before reading.
+__device__ __forceinline__ void fill_factor_table(float* tab, float s_enc)
+{
+    const int c = threadIdx.x;
+    if (c < 128) {
+        float r = 0.0f;
+        if (c != 0 && c != 0x7F) {
+            r = __fdiv_rn(s_enc, e4m3_value(static_cast<uint32_t>(c)));
+            r = r > FLT_MAX ? FLT_MAX : r;
+        }
+        tab[c] = r;
+    }
+}
+
+// Block scale and element factor for a block whose largest magnitude is b:
+// sf = E4M3((b / 6) * S_enc), r = S_enc / sf from the table.
+__device__ __forceinline__ BlockScale block_scale(float b, float s_enc, const float* r_tab)
 {
     BlockScale out;
-    out.sf = e4m3_satfinite(__fmul_rn(__fdiv_rn(b, 6.0f), s_enc));
-    if (out.sf == 0) {
-        out.r = 0.0f;
-    } else {
-        const float r = __fdiv_rn(s_enc, e4m3_value(out.sf));
-        out.r = r > FLT_MAX ? FLT_MAX : r;
-    }
+    out.sf = e4m3_satfinite(__fmul_rn(div6_rn(b), s_enc));
+    out.r = r_tab[out.sf];
     return out;
 }
 

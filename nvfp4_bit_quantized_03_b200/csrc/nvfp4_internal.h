@@ -21,7 +21,8 @@ struct QuantSource {
 struct TileArgs {
     const uint16_t* x;
     int64_t rows, cols, ld;
-    QuantSource src;
+    QuantSource src;      // amax of the row-wise output (of every output outside the dual mode)
+    QuantSource src_col;  // dual mode (row-wise + RHT column-wise): amax of the column output
     uint8_t* row_codes;
     uint8_t* row_scales;
     float* row_amax;
@@ -30,12 +31,18 @@ struct TileArgs {
     float* col_amax;
     uint32_t sign_mask;
     uint64_t seed, offset;
+    uint64_t offset_col;  // dual mode: SR stream of the column output
     int* dev_status;
 };
 
 int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count);
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool rht,
                         uint32_t sign_mask, uint32_t* partials, int grid, cudaStream_t s);
+// One pass for both maxima of the dual mode: amax of RHT(x) along the rows into
+// `partials_rht` and amax of x into `partials_plain` (grid entries each).
+cudaError_t launch_amax_dual(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                             uint32_t sign_mask, uint32_t* partials_rht,
+                             uint32_t* partials_plain, int grid, cudaStream_t s);
 cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                                  const QuantSource& src, float* amax_out0, float* amax_out1,
                                  uint8_t* codes, uint8_t* scales, bool sr, uint64_t seed,

@@ -56,12 +56,16 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
 }
 
 // amax of the random Hadamard transform along the rows: each work item is 16 rows x 4 columns
-// (16 coalesced 8-byte loads), i.e. four 16-element transforms.
+// (16 coalesced 8-byte loads), i.e. four 16-element transforms.  With PLAIN the same loads also
+// give the amax of x itself (the row-wise output of the dual mode).
+template <bool PLAIN>
 __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restrict__ x,
                                                        int64_t rows, int64_t cols, int64_t ld,
                                                        uint32_t sign_mask,
-                                                       uint32_t* __restrict__ partials)
+                                                       uint32_t* __restrict__ partials,
+                                                       uint32_t* __restrict__ partials_plain)
 {
+    uint32_t mp = 0;
     const int64_t cpr = cols >> 2;  // 8-byte column groups per row
     const int64_t total = (rows >> 4) * cpr;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -73,6 +77,11 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
         uint2 v[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) v[k] = __ldg(reinterpret_cast<const uint2*>(base + k * ld));
+        if (PLAIN) {
+#pragma unroll
+            for (int k = 0; k < 16; ++k)
+                mp = __vmaxu2(mp, __vmaxu2(v[k].x & 0x7FFF7FFFu, v[k].y & 0x7FFF7FFFu));
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             float y[16];
@@ -87,6 +96,10 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
         }
     }
     block_max_store(m, partials + blockIdx.x);
+    if (PLAIN) {
+        __syncthreads();  // block_max_store's shared scratch is reused
+        block_max_store(max(mp & 0xFFFFu, mp >> 16) << 16, partials_plain + blockIdx.x);
+    }
 }
 
 // ------------------------------------------------------------------------------------------
@@ -158,13 +171,16 @@ __device__ __forceinline__ uint32_t encode8(const uint4& v, const float* e, cons
 }
 
 template <bool SR>
-__global__ void __launch_bounds__(256) quant_rowwise_kernel(
+__global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, QuantSource src,
     float* amax_out0, float* amax_out1, uint8_t* __restrict__ codes,
     uint8_t* __restrict__ scales, uint64_t seed, uint64_t offset, int* dev_status)
 {
     constexpr int U = 4;
+    __shared__ float r_tab[128];
     const TensorScale ts = fold_amax(src, amax_out0, amax_out1, dev_status);
+    fill_factor_table(r_tab, ts.s_enc);
+    __syncthreads();
     const Philox philox(seed);
     const int lane = threadIdx.x & 31;
     const int64_t cpr = cols >> 3;
@@ -217,7 +233,7 @@ __global__ void __launch_bounds__(256) quant_rowwise_kernel(
 #pragma unroll
             for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(e[j]));
             const float b = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            const BlockScale bs = block_scale(b, ts.s_enc);
+            const BlockScale bs = block_scale(b, ts.s_enc, r_tab);
             uint32_t packed = encode8<SR>(v[u], e, bs, philox, static_cast<uint64_t>(f), offset);
             const uint32_t sf = ts.nonfinite ? 0u : bs.sf;
             if (ts.nonfinite) packed = 0;
@@ -279,8 +295,22 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
     __shared__ float bmax[kTileRows][8];
     __shared__ float tmax[4][8];
 
-    const TensorScale ts = fold_amax(a.src, ROW ? a.row_amax : a.col_amax,
-                                     ROW ? a.col_amax : nullptr, a.dev_status);
+    // Dual mode (row-wise output of x, column-wise output of RHT(x)): each output has its own
+    // amax, hence its own tensor scale, and its own SR stream.  Otherwise one amax serves both.
+    constexpr bool DUAL = ROW && COL && RHT;
+    TensorScale ts_row, ts_col;
+    if (DUAL) {
+        ts_row = fold_amax(a.src, a.row_amax, nullptr, a.dev_status);
+        ts_col = fold_amax(a.src_col, a.col_amax, nullptr, a.dev_status);
+    } else {
+        ts_row = fold_amax(a.src, ROW ? a.row_amax : a.col_amax, ROW ? a.col_amax : nullptr,
+                           a.dev_status);
+        ts_col = ts_row;
+    }
+    __shared__ float r_tab_row[128], r_tab_col[128];
+    fill_factor_table(r_tab_row, ts_row.s_enc);
+    fill_factor_table(r_tab_col, ts_col.s_enc);
+    __syncthreads();
     const Philox philox(a.seed);
     const int t = threadIdx.x;
     const int64_t tiles_c = (a.cols + kTileCols - 1) / kTileCols;
@@ -342,12 +372,12 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float b = BLOCK2D ? tmax[rrow >> 4][rblk + q] : rb[q];
-                const BlockScale bs = block_scale(b, ts.s_enc);
+                const BlockScale bs = block_scale(b, ts_row.s_enc, r_tab_row);
                 const uint64_t e0 = static_cast<uint64_t>(r) * a.cols + c0 + (rblk + q) * 16;
                 encode16<SR>(rv[q], bs, philox, e0, a.offset, words[2 * q], words[2 * q + 1]);
                 sfw |= bs.sf << (8 * q);
             }
-            if (ts.nonfinite) {
+            if (ts_row.nonfinite) {
                 sfw = 0;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) words[q] = 0;
@@ -379,12 +409,12 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
 #pragma unroll
                     for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(y[i]));
                 }
-                const BlockScale bs = block_scale(b, ts.s_enc);
+                const BlockScale bs = block_scale(b, ts_col.s_enc, r_tab_col);
                 const uint64_t e0 = static_cast<uint64_t>(orow) * a.rows + r0 + q * 16;
-                encode16<SR>(y, bs, philox, e0, a.offset, words[2 * q], words[2 * q + 1]);
+                encode16<SR>(y, bs, philox, e0, a.offset_col, words[2 * q], words[2 * q + 1]);
                 sfw |= bs.sf << (8 * q);
             }
-            if (ts.nonfinite) {
+            if (ts_col.nonfinite) {
                 sfw = 0;
 #pragma unroll
                 for (int q = 0; q < 8; ++q) words[q] = 0;
@@ -406,6 +436,18 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
 // Launchers
 // ------------------------------------------------------------------------------------------
 
+// CTAs of `kernel` resident per SM at `threads` threads (no dynamic shared memory); the
+// launchers keep the answer in a function-local static per kernel.
+template <typename Kernel>
+static int resident_ctas(Kernel kernel, int threads)
+{
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess ||
+        n < 1)
+        n = 1;
+    return n;
+}
+
 int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count)
 {
     const int64_t items = rht ? (rows / 16) * (cols / 4) : rows * (cols / 8);
@@ -422,9 +464,19 @@ cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t l
                         uint32_t sign_mask, uint32_t* partials, int grid, cudaStream_t s)
 {
     if (rht)
-        amax_rht_kernel<<<grid, 256, 0, s>>>(x, rows, cols, ld, sign_mask, partials);
+        amax_rht_kernel<false><<<grid, 256, 0, s>>>(x, rows, cols, ld, sign_mask, partials,
+                                                     nullptr);
     else
         amax_kernel<<<grid, 256, 0, s>>>(x, rows, cols, ld, partials);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_amax_dual(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                             uint32_t sign_mask, uint32_t* partials_rht,
+                             uint32_t* partials_plain, int grid, cudaStream_t s)
+{
+    amax_rht_kernel<true><<<grid, 256, 0, s>>>(x, rows, cols, ld, sign_mask, partials_rht,
+                                                partials_plain);
     return cudaGetLastError();
 }
 
@@ -433,9 +485,13 @@ cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, 
                                  uint8_t* codes, uint8_t* scales, bool sr, uint64_t seed,
                                  uint64_t offset, int* dev_status, int sm_count, cudaStream_t s)
 {
+    // One wave of resident CTAs: every CTA folds the amax partials and fills its factor table
+    // once, then strides over the work.
     const int64_t warps = (rows * (cols >> 3) + 127) / 128;
     int64_t grid = (warps + 7) / 8;
-    const int64_t cap = static_cast<int64_t>(sm_count) * 16;
+    static const int resident_sr = resident_ctas(quant_rowwise_kernel<true>, 256);
+    static const int resident_rn = resident_ctas(quant_rowwise_kernel<false>, 256);
+    const int64_t cap = static_cast<int64_t>(sm_count) * (sr ? resident_sr : resident_rn);
     if (grid > cap) grid = cap;
     if (grid < 1) grid = 1;
     if (sr)
@@ -450,9 +506,13 @@ cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, 
 }
 
 template <bool ROW, bool COL, bool B2D, bool RHT, bool SR>
-static void launch_tile_t(const TileArgs& a, int grid, cudaStream_t s)
+static void launch_tile_t(const TileArgs& a, int64_t ntiles, int sm_count, cudaStream_t s)
 {
-    quant_tile_kernel<ROW, COL, B2D, RHT, SR><<<grid, 128, 0, s>>>(a);
+    static const int resident = resident_ctas(quant_tile_kernel<ROW, COL, B2D, RHT, SR>, 128);
+    int64_t grid = static_cast<int64_t>(sm_count) * resident;
+    if (grid > ntiles) grid = ntiles;
+    if (grid < 1) grid = 1;
+    quant_tile_kernel<ROW, COL, B2D, RHT, SR><<<static_cast<int>(grid), 128, 0, s>>>(a);
 }
 
 cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2d, bool rht,
@@ -460,21 +520,20 @@ cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2
 {
     const int64_t ntiles = ((a.rows + kTileRows - 1) / kTileRows) *
                            ((a.cols + kTileCols - 1) / kTileCols);
-    int64_t grid = ntiles;
-    const int64_t cap = static_cast<int64_t>(sm_count) * 16;
-    if (grid > cap) grid = cap;
-    if (grid < 1) grid = 1;
-    const int g = static_cast<int>(grid);
+    const int64_t g = ntiles;
+    const int sm = sm_count;
     // Supported combinations (the API rejects the others before launching).
-    if (row && col && block2d)            launch_tile_t<true, true, true, false, false>(a, g, s);
-    else if (row && !col && block2d)      launch_tile_t<true, false, true, false, false>(a, g, s);
-    else if (!row && col && block2d)      launch_tile_t<false, true, true, false, false>(a, g, s);
-    else if (row && col && !sr)           launch_tile_t<true, true, false, false, false>(a, g, s);
-    else if (row && col && sr)            launch_tile_t<true, true, false, false, true>(a, g, s);
-    else if (col && rht && sr)            launch_tile_t<false, true, false, true, true>(a, g, s);
-    else if (col && rht && !sr)           launch_tile_t<false, true, false, true, false>(a, g, s);
-    else if (col && !rht && sr)           launch_tile_t<false, true, false, false, true>(a, g, s);
-    else if (col && !rht && !sr)          launch_tile_t<false, true, false, false, false>(a, g, s);
+    if (row && col && rht && sr)          launch_tile_t<true, true, false, true, true>(a, g, sm, s);
+    else if (row && col && rht && !sr)    launch_tile_t<true, true, false, true, false>(a, g, sm, s);
+    else if (row && col && block2d)       launch_tile_t<true, true, true, false, false>(a, g, sm, s);
+    else if (row && !col && block2d)      launch_tile_t<true, false, true, false, false>(a, g, sm, s);
+    else if (!row && col && block2d)      launch_tile_t<false, true, true, false, false>(a, g, sm, s);
+    else if (row && col && !sr)           launch_tile_t<true, true, false, false, false>(a, g, sm, s);
+    else if (row && col && sr)            launch_tile_t<true, true, false, false, true>(a, g, sm, s);
+    else if (col && rht && sr)            launch_tile_t<false, true, false, true, true>(a, g, sm, s);
+    else if (col && rht && !sr)           launch_tile_t<false, true, false, true, false>(a, g, sm, s);
+    else if (col && !rht && sr)           launch_tile_t<false, true, false, false, true>(a, g, sm, s);
+    else if (col && !rht && !sr)          launch_tile_t<false, true, false, false, false>(a, g, sm, s);
     else return cudaErrorInvalidValue;
     return cudaGetLastError();
 }
