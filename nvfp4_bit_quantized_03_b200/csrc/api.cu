@@ -193,7 +193,7 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
     }
     a.src_col = src;
     a.sign_mask = sign_mask;
-    a.seed = seed;
+    a.keys = philox_round_keys(seed);
     a.offset = offset;
     a.offset_col = offset;
     a.dev_status = dev_status;
@@ -342,7 +342,7 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
     a.col_scales = static_cast<uint8_t*>(out_col->scales);
     a.col_amax = out_col->amax;
     a.sign_mask = sign_mask;
-    a.seed = seed;
+    a.keys = philox_round_keys(seed);
     a.offset = offset;
     a.offset_col = offset + 1;
     a.dev_status = dev_status;

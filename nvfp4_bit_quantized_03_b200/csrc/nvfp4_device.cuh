@@ -11,6 +11,8 @@
 #include <cstdint>
 #include <cfloat>
 
+#include "nvfp4_internal.h"
+
 namespace nvfp4 {
 
 constexpr uint32_t kDevNonfinite = 1u;  // NVFP4_DEVSTAT_NONFINITE
@@ -42,27 +44,25 @@ __device__ __forceinline__ uint32_t absmax_bits8(const uint4& v)
 // ---- Philox-4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy as 1, 2, 3") ------
 // Ten rounds of the Philox-4x32 bijection: two 32x32 -> 64-bit products by 0xD2511F53 and
 // 0xCD9E8D57 whose halves are xor-ed with the other two words and the round key; the key
-// advances by 0x9E3779B9, 0xBB67AE85 after each round.
+// (seed low, seed high) advances by 0x9E3779B9, 0xBB67AE85 after each round.  The ten round
+// keys depend on the seed alone, so the host computes them (philox_round_keys) and they
+// reach the kernels as launch parameters: each round's xor reads its key from the constant
+// bank instead of recomputing it per call.
 struct Philox {
-    uint32_t k0, k1;
-    __device__ __forceinline__ explicit Philox(uint64_t seed)
-        : k0(static_cast<uint32_t>(seed)), k1(static_cast<uint32_t>(seed >> 32)) {}
+    PhiloxKeys keys;
 
     __device__ __forceinline__ uint4 operator()(uint32_t c0, uint32_t c1, uint32_t c2,
                                                 uint32_t c3) const
     {
-        uint32_t a = k0, b = k1;
 #pragma unroll
         for (int i = 0; i < 10; ++i) {
             // one 32 x 32 -> 64-bit product per multiplier gives both halves
             const uint64_t p0 = static_cast<uint64_t>(c0) * 0xD2511F53u;
             const uint64_t p1 = static_cast<uint64_t>(c2) * 0xCD9E8D57u;
-            c0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ a;
+            c0 = static_cast<uint32_t>(p1 >> 32) ^ c1 ^ keys.k0[i];
             c1 = static_cast<uint32_t>(p1);
-            c2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ b;
+            c2 = static_cast<uint32_t>(p0 >> 32) ^ c3 ^ keys.k1[i];
             c3 = static_cast<uint32_t>(p0);
-            a += 0x9E3779B9u;
-            b += 0xBB67AE85u;
         }
         return make_uint4(c0, c1, c2, c3);
     }

@@ -12,6 +12,25 @@ constexpr int kMaxPartials = 2048;
 
 // Where a quantize kernel gets the tensor amax from: the partial maxima written by the
 // amax pass (FP32 bit patterns), or a caller-given FP32 value.
+// The ten Philox-4x32-10 round keys of a seed: round i uses (seed low + i * 0x9E3779B9,
+// seed high + i * 0xBB67AE85).
+struct PhiloxKeys {
+    uint32_t k0[10], k1[10];
+};
+
+inline PhiloxKeys philox_round_keys(uint64_t seed)
+{
+    PhiloxKeys k;
+    uint32_t a = static_cast<uint32_t>(seed), b = static_cast<uint32_t>(seed >> 32);
+    for (int i = 0; i < 10; ++i) {
+        k.k0[i] = a;
+        k.k1[i] = b;
+        a += 0x9E3779B9u;
+        b += 0xBB67AE85u;
+    }
+    return k;
+}
+
 struct QuantSource {
     const uint32_t* partials;
     int n_partials;
@@ -30,7 +49,8 @@ struct TileArgs {
     uint8_t* col_scales;
     float* col_amax;
     uint32_t sign_mask;
-    uint64_t seed, offset;
+    PhiloxKeys keys;      // round keys of the SR seed
+    uint64_t offset;
     uint64_t offset_col;  // dual mode: SR stream of the column output
     int* dev_status;
 };

@@ -174,14 +174,14 @@ template <bool SR>
 __global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
     const uint16_t* __restrict__ x, int64_t rows, int64_t cols, int64_t ld, QuantSource src,
     float* amax_out0, float* amax_out1, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ scales, uint64_t seed, uint64_t offset, int* dev_status)
+    uint8_t* __restrict__ scales, const PhiloxKeys keys, uint64_t offset, int* dev_status)
 {
     constexpr int U = 4;
     __shared__ float r_tab[128];
     const TensorScale ts = fold_amax(src, amax_out0, amax_out1, dev_status);
     fill_factor_table(r_tab, ts.s_enc);
     __syncthreads();
-    const Philox philox(seed);
+    const Philox philox{keys};
     const int lane = threadIdx.x & 31;
     const int64_t cpr = cols >> 3;
     const int64_t gpr = cols >> 6;
@@ -289,7 +289,7 @@ __device__ __forceinline__ void encode16(const float* y, const BlockScale& bs, c
 }
 
 template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR>
-__global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
+__global__ void __launch_bounds__(128, SR ? 6 : 8) quant_tile_kernel(TileArgs a)
 {
     __shared__ __align__(16) uint16_t tile[kTileRows * kTilePitch];
     __shared__ float bmax[kTileRows][8];
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
     fill_factor_table(r_tab_row, ts_row.s_enc);
     fill_factor_table(r_tab_col, ts_col.s_enc);
     __syncthreads();
-    const Philox philox(a.seed);
+    const Philox philox{a.keys};
     const int t = threadIdx.x;
     const int64_t tiles_c = (a.cols + kTileCols - 1) / kTileCols;
     const int64_t tiles_r = (a.rows + kTileRows - 1) / kTileRows;
@@ -334,26 +334,25 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
         }
         __syncthreads();
 
-        // Row walk: thread t -> row t % 64, blocks 4 (t / 64) .. +3.
+        // Row walk: thread t -> row t % 64, blocks 4 (t / 64) .. +3.  One 16-value block is
+        // held in registers at a time (re-read from shared memory when it is encoded).
         const int rrow = t & 63, rblk = (t >> 6) * 4;
-        float rv[4][16];
-        float rb[4];
-        if (ROW || BLOCK2D) {
+        auto load_row_block = [&](int q, float* v) {
+            const uint16_t* src = tile + rrow * kTilePitch + (rblk + q) * 16;
+            unpack8(*reinterpret_cast<const uint4*>(src), v);
+            unpack8(*reinterpret_cast<const uint4*>(src + 8), v + 8);
+        };
+        if (BLOCK2D) {
+            // 16x16 tile maxima: row-block maxima, then the column of 16 of them per tile
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const uint16_t* src = tile + rrow * kTilePitch + (rblk + q) * 16;
-                const uint4 lo = *reinterpret_cast<const uint4*>(src);
-                const uint4 hi = *reinterpret_cast<const uint4*>(src + 8);
-                unpack8(lo, rv[q]);
-                unpack8(hi, rv[q] + 8);
+                float v[16];
+                load_row_block(q, v);
                 float m = 0.0f;
 #pragma unroll
-                for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(rv[q][j]));
-                rb[q] = m;
-                if (BLOCK2D) bmax[rrow][rblk + q] = m;
+                for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
+                bmax[rrow][rblk + q] = m;
             }
-        }
-        if (BLOCK2D) {
             __syncthreads();
             if (t < 32) {
                 const int tr = t >> 3, tc = t & 7;
@@ -371,10 +370,19 @@ __global__ void __launch_bounds__(128) quant_tile_kernel(TileArgs a)
             uint32_t sfw = 0;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const float b = BLOCK2D ? tmax[rrow >> 4][rblk + q] : rb[q];
+                float rv[16];
+                load_row_block(q, rv);
+                float b;
+                if (BLOCK2D) {
+                    b = tmax[rrow >> 4][rblk + q];
+                } else {
+                    b = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) b = fmaxf(b, fabsf(rv[j]));
+                }
                 const BlockScale bs = block_scale(b, ts_row.s_enc, r_tab_row);
                 const uint64_t e0 = static_cast<uint64_t>(r) * a.cols + c0 + (rblk + q) * 16;
-                encode16<SR>(rv[q], bs, philox, e0, a.offset, words[2 * q], words[2 * q + 1]);
+                encode16<SR>(rv, bs, philox, e0, a.offset, words[2 * q], words[2 * q + 1]);
                 sfw |= bs.sf << (8 * q);
             }
             if (ts_row.nonfinite) {
@@ -453,7 +461,13 @@ int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count)
     const int64_t items = rht ? (rows / 16) * (cols / 4) : rows * (cols / 8);
     const int64_t per_cta = rht ? 256 : 256 * 4;
     int64_t g = (items + per_cta - 1) / per_cta;
-    const int64_t cap = static_cast<int64_t>(sm_count) * 8;
+    // one wave of resident CTAs (the amax passes are short; a partial second wave is a tail)
+    static const int resident_plain = resident_ctas(amax_kernel, 256);
+    static const int resident_rht = resident_ctas(amax_rht_kernel<false>, 256) <
+                                            resident_ctas(amax_rht_kernel<true>, 256)
+                                        ? resident_ctas(amax_rht_kernel<false>, 256)
+                                        : resident_ctas(amax_rht_kernel<true>, 256);
+    const int64_t cap = static_cast<int64_t>(sm_count) * (rht ? resident_rht : resident_plain);
     if (g > cap) g = cap;
     if (g > kMaxPartials) g = kMaxPartials;
     if (g < 1) g = 1;
@@ -489,6 +503,7 @@ cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, 
     // once, then strides over the work.
     const int64_t warps = (rows * (cols >> 3) + 127) / 128;
     int64_t grid = (warps + 7) / 8;
+    const PhiloxKeys keys = philox_round_keys(seed);
     static const int resident_sr = resident_ctas(quant_rowwise_kernel<true>, 256);
     static const int resident_rn = resident_ctas(quant_rowwise_kernel<false>, 256);
     const int64_t cap = static_cast<int64_t>(sm_count) * (sr ? resident_sr : resident_rn);
@@ -496,11 +511,11 @@ cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, 
     if (grid < 1) grid = 1;
     if (sr)
         quant_rowwise_kernel<true><<<static_cast<int>(grid), 256, 0, s>>>(
-            x, rows, cols, ld, src, amax_out0, amax_out1, codes, scales, seed, offset,
+            x, rows, cols, ld, src, amax_out0, amax_out1, codes, scales, keys, offset,
             dev_status);
     else
         quant_rowwise_kernel<false><<<static_cast<int>(grid), 256, 0, s>>>(
-            x, rows, cols, ld, src, amax_out0, amax_out1, codes, scales, seed, offset,
+            x, rows, cols, ld, src, amax_out0, amax_out1, codes, scales, keys, offset,
             dev_status);
     return cudaGetLastError();
 }
