@@ -7,8 +7,11 @@
 // Design (one CTA per SM, persistent over 128 x 256 output tiles, 22 warps):
 //   warp 0      TMA producer: per 256-wide K block, the A (128 x 128 B) and B (256 x 128 B)
 //               code tiles with 128-byte swizzle, plus the block scales (contiguous 512-byte
-//               tiles of the MMA scale layout) by bulk copies; a 3-stage shared-memory ring
-//               guarded by mbarriers.
+//               tiles of the MMA scale layout) by bulk copies; a shared-memory ring of 4
+//               stages (bf16 output) or 3 (FP32 output) guarded by mbarriers.  One stage's
+//               round trip (TMA ~1.7 k cycles, scale staging ~0.55 k, issue ~0.5 k, MMAs +
+//               release ~1.1 k) is about four stages of MMA work, so with three stages the
+//               tensor pipe idles about a third of the time.
 //   warps 2-5   scale stagers, one per 32-lane quarter of tensor memory: move each stage's
 //               scales shared -> registers -> tensor memory (ld.shared + tcgen05.st, into a
 //               per-stage column range), so the tensor pipe never spends time on scale copies.
@@ -18,9 +21,9 @@
 //   warps 6-21  epilogue: each warp drains one 32-lane quarter x 64 columns of the
 //               accumulator into registers (tcgen05.ld), releases the accumulator so the
 //               next tile's MMAs start at once, then scales by 1 / (S_enc,A S_enc,B) and
-//               writes FP32 or bf16 rows through a 64-byte-swizzled shared-memory staging
-//               buffer with TMA bulk tensor stores (whole 64-byte row segments, clipped at the
-//               matrix edge) while the next tile computes.
+//               writes FP32 or bf16 rows through a per-warp shared-memory staging buffer
+//               with paced TMA bulk tensor stores (clipped at the matrix edge) while the next
+//               tile computes.
 // Every wait on an mbarrier is bounded in time; on expiry the kernel records
 // NVFP4_DEVSTAT_TIMEOUT, drains its in-flight copies and MMAs (again with a limit), frees
 // its tensor memory and returns.
@@ -42,7 +45,6 @@ constexpr int BM = 128;                 // tile rows (A rows, TMEM lanes)
 constexpr int BN = 256;                 // tile columns (B rows, accumulator columns)
 constexpr int BK = 256;                 // K elements per pipeline stage (128 bytes per row)
 constexpr int MMA_K = 64;               // K per tcgen05.mma of kind::mxf4nvf4
-constexpr int STAGES = 3;
 constexpr int A_BYTES = BM * BK / 2;    // 16 KB
 constexpr int B_BYTES = BN * BK / 2;    // 32 KB
 constexpr int SF_TILE = 512;            // 128 rows x 4 blocks of scales
@@ -58,15 +60,36 @@ constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;              // accumulator: columns [0, 256)
 constexpr int SF_COL = BN;              // scales: 48 columns per stage from column 256
 constexpr int SF_COLS_PER_STAGE = (BK / MMA_K) * (4 + 8);
-constexpr int STAGING_BYTES = 2048;     // per epilogue warp: 32 rows x 64 bytes of output
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + NUM_EPI_WARPS * STAGING_BYTES + BAR_BYTES + 1024;
-static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+
+// Pipeline shape per output type.  A bf16 tile (64 KB of output) goes out through 512-byte
+// staging buffers, which leaves room for a fourth operand stage; an FP32 tile (128 KB) keeps
+// 2 KB buffers and three stages.  The epilogue's TMA stores are paced (a first-round delay and
+// a gap between rounds) so that they do not crowd the next tile's first operand loads.
+template <bool BF16>
+struct Pipe {
+    static constexpr int STAGES = BF16 ? 4 : 3;
+    static constexpr int STAGING_BYTES = BF16 ? 512 : 2048;  // per epilogue warp
+    static constexpr int SMEM_BYTES =
+        STAGES * STAGE_BYTES + NUM_EPI_WARPS * STAGING_BYTES + BAR_BYTES + 1024;
+    static constexpr unsigned FIRST_NS = BF16 ? 3000u : 0u;
+    static constexpr unsigned GAP_NS = BF16 ? 1000u : 2000u;
+    // shared-memory barrier slots
+    static constexpr int BAR_FULL = 0;                     // [STAGES] TMA bytes of a stage landed
+    static constexpr int BAR_EMPTY = BAR_FULL + STAGES;    // [STAGES] the stage's MMAs completed
+    static constexpr int BAR_SF = BAR_EMPTY + STAGES;      // [STAGES] the stage's scales are in TMEM
+    static constexpr int BAR_ACC_FULL = BAR_SF + STAGES;   // the tile's accumulator is complete
+    static constexpr int BAR_ACC_EMPTY = BAR_ACC_FULL + 1; // the epilogue drained the accumulator
+    static constexpr int BAR_DRAIN = BAR_ACC_EMPTY + 1;    // teardown after an abort
+    static constexpr int NUM_BARS = BAR_DRAIN + 1;
+    static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+    static_assert(NUM_BARS * 8 + 16 <= BAR_BYTES, "barrier area");
+    static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "tensor memory budget");
+};
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait
 constexpr int kDevTimeoutBit = 2;       // NVFP4_DEVSTAT_TIMEOUT
 
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
-static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "tensor memory budget");
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format 1), both
 // K-major, UE4M3 scales (bit 23 = 0), N >> 3 at bit 17, M >> 4 at bit 24, dense K = 64.
@@ -275,29 +298,38 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 }
 
 // One epilogue warp's 32 x 64 slice of the tile (row `lane`, values v[0..63] in FP32 bits) to
-// global memory: scaled by alpha, converted, written as 32 x 64-byte boxes into the warp's
-// staging buffer and sent with TMA bulk tensor stores (bf16: 2 boxes of 32 columns; FP32: 4
-// boxes of 16).  Row `lane` of a box sits at lane * 64 with its four 16-byte chunks permuted
-// by the 64-byte swizzle (chunk c at c ^ ((row / 2) % 4)), which the tensor map undoes.
+// global memory, scaled by alpha and converted, through the warp's staging buffer with TMA bulk
+// tensor stores.
+//  * bf16: 8 rounds of 16 bytes (8 columns) of every row, boxes of 32 rows x 16 bytes; row
+//    `lane` of a box sits at lane * 16, so the warp's 16-byte shared stores are conflict-free.
+//  * FP32: 4 rounds of 64 bytes (16 columns), boxes of 32 rows x 64 bytes; row `lane` sits at
+//    lane * 64 with its four 16-byte chunks permuted by the 64-byte swizzle (chunk c at
+//    c ^ ((row / 2) % 4)), which the tensor map undoes.
+// Each round waits only for the previous box to leave the buffer; rounds are paced by
+// Pipe::FIRST_NS / GAP_NS.
 template <bool BF16>
 __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint32_t stage_buf,
                                             int lane, const CUtensorMap* tmap_d, int n0, int y,
                                             int M, int N)
 {
-    constexpr int COLS = BF16 ? 32 : 16;  // columns per 64-byte box row
-    const uint32_t row_base = stage_buf + 64 * lane;
-    const uint32_t swz = (lane >> 1) & 3;
+    using P = Pipe<BF16>;
+    constexpr int CHUNKS = BF16 ? 1 : 4;             // 16-byte chunks per box row
+    constexpr int COLS = CHUNKS * (BF16 ? 8 : 4);    // columns per box row
+    const uint32_t row_base = stage_buf + 16 * CHUNKS * lane;
+    const uint32_t swz = BF16 ? 0u : ((lane >> 1) & 3);
 #pragma unroll
     for (int r = 0; r < 64 / COLS; ++r) {
+        if (r == 0 && P::FIRST_NS) __nanosleep(P::FIRST_NS);
+        if (r != 0 && P::GAP_NS) __nanosleep(P::GAP_NS);
         if (lane == 0) bulk_wait_read();  // the previous box has left the buffer
         __syncwarp();
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < CHUNKS; ++c) {
             uint32_t o[4];
             if (BF16) {
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    const int j = r * 32 + c * 8 + 2 * h;
+                    const int j = r * 8 + 2 * h;
                     const __nv_bfloat162 b2 =
                         __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j]), alpha),
                                               __fmul_rn(__uint_as_float(v[j + 1]), alpha));
@@ -319,21 +351,17 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint
     }
 }
 
-// Shared-memory barrier slots.
-constexpr int BAR_FULL = 0;                 // [STAGES] TMA bytes of a stage landed
-constexpr int BAR_EMPTY = BAR_FULL + STAGES;    // [STAGES] the stage's MMAs completed
-constexpr int BAR_SF = BAR_EMPTY + STAGES;      // [STAGES] the stage's scales are in TMEM
-constexpr int BAR_ACC_FULL = BAR_SF + STAGES;   // the tile's accumulator is complete
-constexpr int BAR_ACC_EMPTY = BAR_ACC_FULL + 1; // the epilogue drained the accumulator
-constexpr int BAR_DRAIN = BAR_ACC_EMPTY + 1;    // teardown after an abort
-constexpr int NUM_BARS = BAR_DRAIN + 1;
-static_assert(NUM_BARS * 8 + 16 <= BAR_BYTES, "barrier area");
-
+template <bool BF16>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_d, const Params p)
 {
+    using P = Pipe<BF16>;
+    constexpr int STAGES = P::STAGES, STAGING_BYTES = P::STAGING_BYTES;
+    constexpr int BAR_FULL = P::BAR_FULL, BAR_EMPTY = P::BAR_EMPTY, BAR_SF = P::BAR_SF;
+    constexpr int BAR_ACC_FULL = P::BAR_ACC_FULL, BAR_ACC_EMPTY = P::BAR_ACC_EMPTY;
+    constexpr int BAR_DRAIN = P::BAR_DRAIN, NUM_BARS = P::NUM_BARS;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -555,10 +583,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tile_coords(t, tiles_m, tiles_n, tm, tn);
             const int y = tm * BM + 32 * q;       // first output row of this warp's slice
             const int n0 = tn * BN + 64 * chunk;  // first output column
-            if (p.out_bf16)
-                store_slice<true>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
-            else
-                store_slice<false>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
+            store_slice<BF16>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
         }
         if (lane == 0) bulk_wait_all();
     }
@@ -606,8 +631,9 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// 2D map over D (rows x N elements, row stride ldd), boxes of 32 rows x 64 bytes with
-// 64-byte swizzle, for the epilogue's bulk tensor stores.
+// 2D map over D (rows x N elements, row stride ldd) for the epilogue's bulk tensor stores
+// (the map clips rows beyond M): bf16 boxes of 32 rows x 16 bytes, unswizzled; FP32 boxes of
+// 32 rows x 64 bytes with the 64-byte swizzle.
 bool make_output_map(CUtensorMap* map, void* D, int64_t M, int64_t N, int64_t ldd, bool bf16)
 {
     auto enc = tensor_map_encoder();
@@ -615,10 +641,11 @@ bool make_output_map(CUtensorMap* map, void* D, int64_t M, int64_t N, int64_t ld
     const int64_t esize = bf16 ? 2 : 4;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldd * esize)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / esize), 32};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>((bf16 ? 16 : 64) / esize), 32};
     const cuuint32_t estr[2] = {1, 1};
     return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, D,
-               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+               dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               bf16 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B,
                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -630,8 +657,13 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        const cudaError_t e = cudaFuncSetAttribute(
-            gemm_nvf4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             Pipe<true>::SMEM_BYTES);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(gemm_nvf4_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Pipe<false>::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
@@ -653,7 +685,10 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     p.dev_status = g.dev_status;
     const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < sm_count ? tiles : sm_count);
-    gemm_nvf4_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(ma, mb, md, p);
+    if (g.out_bf16)
+        gemm_nvf4_kernel<true><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
+    else
+        gemm_nvf4_kernel<false><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, md, p);
     return cudaGetLastError();
 }
 
