@@ -53,6 +53,12 @@ def lib():
         L.nvo_e2m1_rtn_many.argtypes, L.nvo_e2m1_rtn_many.restype = [vp, i64, vp], None
         L.nvo_e2m1_sr_many.argtypes, L.nvo_e2m1_sr_many.restype = [vp, vp, i64, vp], None
         L.nvo_e4m3_many.argtypes, L.nvo_e4m3_many.restype = [vp, i64, vp], None
+        L.nvo_mx_exponent.argtypes, L.nvo_mx_exponent.restype = [fp], ctypes.c_int
+        L.nvo_e8m0_decode.argtypes, L.nvo_e8m0_decode.restype = [u8], dp
+        L.nvo_mx_quantize.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, u16,
+                                      ctypes.c_int, u64, u64, vp, vp]
+        L.nvo_mx_quantize.restype = ctypes.c_int
+        L.nvo_mx_dequantize.argtypes, L.nvo_mx_dequantize.restype = [vp, vp, i64, i64, vp], None
         _lib = L
     return _lib
 
@@ -182,6 +188,54 @@ def quantize(x_bf16: np.ndarray, *, transpose=False, rht=False, sign_mask=0, blo
     return Quantized(codes, scales, amax_out.value, st)
 
 
+# ---- MXFP4, the comparison format ------------------------------------------------------
+
+class MXQuantized:
+    """An MXFP4 operand in the oracle's plain layout: codes [R x C/2] as NVFP4, scales
+    [R x C/32] E8M0 bytes row-major (scale = 2^(byte - 127)); no tensor scale."""
+
+    def __init__(self, codes, scales, status):
+        self.codes, self.scales, self.status = codes, scales, status
+
+    @property
+    def rows(self):
+        return self.codes.shape[0]
+
+    @property
+    def cols(self):
+        return self.codes.shape[1] * 2
+
+    def dequantize(self) -> np.ndarray:
+        R, C = self.rows, self.cols
+        out = np.zeros((R, C), dtype=np.float64)
+        lib().nvo_mx_dequantize(_ptr(self.codes), _ptr(self.scales), R, C, _ptr(out))
+        return out
+
+
+def mx_exponent(b: float) -> int:
+    return lib().nvo_mx_exponent(b)
+
+
+def e8m0_decode(code: int) -> float:
+    return lib().nvo_e8m0_decode(code)
+
+
+def mx_quantize(x_bf16: np.ndarray, *, transpose=False, rht=False, sign_mask=0, sr=False,
+                seed=0, offset=0) -> MXQuantized:
+    """MXFP4-quantize the bf16 matrix ``x_bf16`` along its rows (or, with ``transpose``,
+    quantize x^T), in blocks of 32 with E8M0 power-of-two scales."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    R, C = (cols, rows) if transpose else (rows, cols)
+    codes = np.zeros((R, C // 2), dtype=np.uint8)
+    scales = np.zeros((R, C // 32), dtype=np.uint8)
+    st = lib().nvo_mx_quantize(_ptr(x), rows, cols, cols, int(transpose), int(rht), sign_mask,
+                               int(sr), seed, offset, _ptr(codes), _ptr(scales))
+    if st not in (NVO_OK, NVO_ERR_NONFINITE):
+        raise ValueError(f"oracle MX quantize rejected the arguments (status {st})")
+    return MXQuantized(codes, scales, st)
+
+
 def gemm_ref_loop(A: np.ndarray, B: np.ndarray) -> np.ndarray:
     """D = A . B^T by the plain FP64 triple loop (tiny shapes only)."""
     A = np.ascontiguousarray(A, dtype=np.float64)
@@ -200,7 +254,7 @@ def row_norms(A: np.ndarray) -> np.ndarray:
     return out
 
 
-def gemm_ref(qa: Quantized, qb: Quantized, rows=None, cols=None):
+def gemm_ref(qa, qb, rows=None, cols=None):
     """Reference D = deq(A) . deq(B)^T in FP64 (numpy matmul as the dot-product step) and
     the normaliser ||A[m,:]|| * ||B[n,:]|| for each entry, optionally restricted to the
     sampled output rows and columns."""

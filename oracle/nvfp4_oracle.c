@@ -377,6 +377,92 @@ int nvo_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
     return NVO_OK;
 }
 
+/* ------------------------------------------------------------------------------------
+ * MXFP4, the comparison format of [P1 Formato NVFP4] (blocks of 32 elements, where NVFP4
+ * uses 16) and of [P1 Nuevo Formato NVFP4] (MX scale factors are coarser than E4M3).
+ * [MX] defines it: E2M1 elements in blocks of 32 sharing one scale X = 2^E stored as an
+ * E8M0 byte (the unsigned exponent E + 127; 255 is NaN), and no per-tensor scale.  For a
+ * block whose largest magnitude is b, E = floor(log2(b)) - 2, 2 being the exponent of the
+ * largest power of two E2M1 holds (4); E is clamped to E8M0's range [-127, 127].  Each
+ * element becomes E2M1(V / X), rounded to nearest even and saturating at 6 ([MX] clamps
+ * values beyond the element format's largest normal).
+ * READING: a block of zeros gets E = -127 (code 0); its codes are 0 whatever E is.
+ * ---------------------------------------------------------------------------------- */
+int nvo_mx_exponent(float b)
+{
+    if (!(b > 0.0f)) return -127;
+    int e;
+    frexpf(b, &e); /* b = m * 2^e with m in [0.5, 1): floor(log2(b)) = e - 1, exactly */
+    int x = (e - 1) - 2;
+    if (x < -127) x = -127;
+    if (x > 127) x = 127;
+    return x;
+}
+
+double nvo_e8m0_decode(uint8_t code) { return ldexp(1.0, (int)code - 127); }
+
+/* MXFP4 quantization of the logical matrix L (x, or x^T with `transpose`) along its rows,
+ * in blocks of 32: codes as nvo_quantize, scales R' x (C' / 32) E8M0 bytes row-major.
+ * sr: stochastic rounding of V / X with element index e = r * C' + c of L (the same bits
+ * as the NVFP4 path; READING: the MX variant reuses the recipe's rounding choices).
+ * Non-finite data anywhere in L: codes and scales 0, NVO_ERR_NONFINITE. */
+int nvo_mx_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                    int transpose, int rht, uint16_t sign_mask, int sr, uint64_t seed,
+                    uint64_t offset, uint8_t* codes, uint8_t* scales)
+{
+    int64_t Rl = transpose ? cols : rows;
+    int64_t Cl = transpose ? rows : cols;
+    if (Rl <= 0 || Cl <= 0 || (Cl % 32) != 0) return NVO_ERR_ARG;
+    int64_t nb = Cl / 32;
+    memset(codes, 0, (size_t)(Rl * Cl / 2));
+    memset(scales, 0, (size_t)(Rl * nb));
+    float* row = (float*)malloc(sizeof(float) * (size_t)Cl);
+    if (!row) return NVO_ERR_ARG;
+    for (int64_t r = 0; r < Rl; ++r) {
+        build_rows(x, ld, transpose, rht, sign_mask, r, 1, Cl, row);
+        for (int64_t c = 0; c < Cl; ++c)
+            if (!isfinite(row[c])) {
+                free(row);
+                memset(codes, 0, (size_t)(Rl * Cl / 2));
+                memset(scales, 0, (size_t)(Rl * nb));
+                return NVO_ERR_NONFINITE;
+            }
+        for (int64_t kb = 0; kb < nb; ++kb) {
+            const float* blk = row + kb * 32;
+            float b = 0.0f;
+            for (int c = 0; c < 32; ++c)
+                if (fabsf(blk[c]) > b) b = fabsf(blk[c]);
+            int E = nvo_mx_exponent(b);
+            scales[r * nb + kb] = (uint8_t)(E + 127);
+            for (int c = 0; c < 32; ++c) {
+                float v = ldexpf(blk[c], -E); /* V / 2^E, one correctly rounded scaling */
+                int64_t col = kb * 32 + c;
+                uint8_t q;
+                if (sr) q = nvo_e2m1_sr(v, nvo_sr_bits(seed, offset, (uint64_t)(r * Cl + col)));
+                else q = nvo_e2m1_rtn(v);
+                uint8_t* byte = codes + (r * Cl + col) / 2;
+                if (col & 1) *byte = (uint8_t)((*byte & 0x0Fu) | (q << 4));
+                else *byte = (uint8_t)((*byte & 0xF0u) | q);
+            }
+        }
+    }
+    free(row);
+    return NVO_OK;
+}
+
+/* Dequantized MXFP4 values: e2m1(code) * 2^(scale - 127), in FP64. */
+void nvo_mx_dequantize(const uint8_t* codes, const uint8_t* scales, int64_t R, int64_t C,
+                       double* out)
+{
+    int64_t nb = C / 32;
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t c = 0; c < C; ++c) {
+            uint8_t byte = codes[(r * C + c) / 2];
+            uint8_t q = (c & 1) ? (uint8_t)(byte >> 4) : (uint8_t)(byte & 0xF);
+            out[r * C + c] = nvo_e2m1_decode(q) * nvo_e8m0_decode(scales[r * nb + c / 32]);
+        }
+}
+
 /* Dequantized value of every element: e2m1(code) * float(sf) / S_enc, in FP64. */
 void nvo_dequantize(const uint8_t* codes, const uint8_t* scales, float amax,
                     int64_t R, int64_t C, double* out)
