@@ -29,6 +29,13 @@ import synth  # noqa: E402
 
 METRIC = "NVFP4 GEMM TFLOPS & quantize GB/s on 1 B200, % of FP4/HBM roofline"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2.25 PFLOP/s)
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the bf16-output GEMM at the
+# MLP's shapes (8192 x 20480 x 5120), from
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none \
+#       -k regex:gemm_nvf4 -s 2 -c 1 python bench.py --kernel gemm --steps 2 --warmup 3
+# (295,237,632 read + 309,510,400 written; the algorithmic bytes are ~415 MB: each A row tile
+# is read by 80 column tiles and each B tile by 64 row tiles, mostly from L2).
+GEMM_BF16_DRAM_BYTES = 604_748_032
 
 
 def _peaks():
@@ -388,8 +395,14 @@ def run_ours(args):
     gemm_ms = [a.elapsed_time(b) for a, b in events["gemm"]]
     quant_ms = [a.elapsed_time(b) for a, b in events["quant"]]
     gemm_avg_ms = sum(gemm_ms) / len(gemm_ms)
+    # the step's GEMMs come as (fprop, dgrad, wgrad) per linear: bf16, bf16, FP32 outputs.
+    # The roofline object describes the dominant kernel, the bf16-output instantiation.
+    bf16_ms = [t for i, t in enumerate(gemm_ms) if i % 3 != 2]
+    f32_ms = [t for i, t in enumerate(gemm_ms) if i % 3 == 2]
+    bf16_avg_ms = sum(bf16_ms) / len(bf16_ms)
+    f32_avg_ms = sum(f32_ms) / len(f32_ms)
     flops_per_launch = step.flops_per_gemm[0]  # every GEMM of this workload: 2*8192*5120*20480
-    achieved = flops_per_launch / (gemm_avg_ms / 1e3) / 1e12
+    achieved = flops_per_launch / (bf16_avg_ms / 1e3) / 1e12
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     quant_gbs = step.quant_bytes() * args.steps / (sum(quant_ms) / 1e3) / 1e9
 
@@ -435,11 +448,15 @@ def run_ours(args):
                        "l2": "inputs larger than L2: 1.26 GB of bf16 inputs read per step",
                        "parallelism": "replicas" if world > 1 else "single GPU"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp4_peak,
-                         "unit": "TFLOP/s", "frac": achieved / fp4_peak, "traffic": None,
-                         "kernel": "gemm_nvf4_kernel",
+                         "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                         "traffic": GEMM_BF16_DRAM_BYTES,
+                         "kernel": "gemm_nvf4_kernel<bf16 out> (fprop and dgrad, 4 of 6 GEMMs)",
                          "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} "
                                         f"TFLOP/s x {FP4_OVER_BF16:g} (nominal FP4:BF16)",
-                         "avg_launch_ms": gemm_avg_ms},
+                         "avg_launch_ms": bf16_avg_ms,
+                         "all_gemms_avg_launch_ms": gemm_avg_ms,
+                         "fp32_out_gemm_avg_launch_ms": f32_avg_ms,
+                         "fp32_out_gemm_tflops": flops_per_launch / (f32_avg_ms / 1e3) / 1e12},
             "quantize": {"gbps": quant_gbs, "peak_gbs": peaks["hbm_gbs"],
                          "frac": quant_gbs / peaks["hbm_gbs"],
                          "bytes_per_step": step.quant_bytes(),
@@ -595,6 +612,67 @@ def run_sweep(args):
     return 0
 
 
+def run_dense8b(args):
+    """8B-class dense transformer layer stack at tokens 16384, d 4096: four layers whose five
+    linears (QKV 4096->6144, O 4096->4096, gate and up 4096->14336, down 14336->4096) run
+    fprop + dgrad + wgrad with the full NVFP4 recipe, and a final layer whose linears stay bf16
+    (the pages' selective-precision policy), run as torch bf16 matmuls (cuBLAS) and timed apart.
+    The four NVFP4 layers share one set of synthetic inputs: their work is identical.  Prints
+    one JSON line (not the benchmark's headline line)."""
+    import torch
+    wl = synth.dense_8b_layer()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    step = Step(wl, dev)
+    layers = 4
+
+    def bf16_layer():
+        for L in step.layers:
+            X, W, dY = L["X"], L["W"], L["dY"]
+            torch.matmul(X, W.t(), out=L["bf16_out"][0])
+            torch.matmul(dY, W, out=L["bf16_out"][1])
+            torch.matmul(dY.t(), X, out=L["bf16_out"][2])
+
+    for L in step.layers:
+        T, I, O = L["lin"].T, L["lin"].I, L["lin"].O
+        L["bf16_out"] = (torch.empty((T, O), dtype=torch.bfloat16, device=dev),
+                         torch.empty((T, I), dtype=torch.bfloat16, device=dev),
+                         torch.empty((O, I), dtype=torch.bfloat16, device=dev))
+    for _ in range(args.warmup):
+        for _ in range(layers):
+            step.run()
+        bf16_layer()
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    nv_ms = bf_ms = 0.0
+    for _ in range(args.steps):
+        ev[0].record()
+        for _ in range(layers):
+            step.run()
+        ev[1].record()
+        bf16_layer()
+        ev[2].record()
+        torch.cuda.synchronize()
+        nv_ms += ev[0].elapsed_time(ev[1])
+        bf_ms += ev[1].elapsed_time(ev[2])
+    nv_ms /= args.steps
+    bf_ms /= args.steps
+    flops_layer = step.gemm_flops
+    st = int(step.dev_status.item())
+    print(json.dumps({
+        "workload": wl.name, "steps": args.steps, "warmup": args.warmup,
+        "nvfp4_layers": layers, "nvfp4_ms_per_step": nv_ms,
+        "nvfp4_tflops": layers * flops_layer / (nv_ms / 1e3) / 1e12,
+        "nvfp4_tflop_per_step": layers * flops_layer / 1e12,
+        "bf16_layer_ms": bf_ms, "bf16_tflops": flops_layer / (bf_ms / 1e3) / 1e12,
+        "bf16_share_of_step": bf_ms / (nv_ms + bf_ms),
+        "recipe": "NVFP4 layers: W 16x16 RTN, X 1x16 RTN + RHT16 col, dY 1x16 SR + RHT16 SR col; "
+                  "bf16 layer: torch.matmul (cuBLAS), no quantization",
+        "data": "synthetic, seed 4: activations N(0,1) with 1% x50, weights N(0,0.02), "
+                "gradients N(0,1e-3) with 0.5% x100; one input set shared by the 4 NVFP4 layers",
+        "dev_status": st}), flush=True)
+    return 0 if st == 0 else 1
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -609,6 +687,9 @@ def main(argv=None):
                     help="quantizer bandwidth sweep over 2^n-element tensors (one line per point)")
     ap.add_argument("--sweep-min", type=int, default=20)
     ap.add_argument("--sweep-max", type=int, default=30)
+    ap.add_argument("--workload", choices=["mlp12b", "dense8b"], default="mlp12b",
+                    help="dense8b: the 8B-class layer stack (4 NVFP4 layers + 1 bf16 layer), "
+                         "reported on its own JSON line")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)  # at least 3 untimed warm-up steps
     if args.impl == "reference":
@@ -617,6 +698,8 @@ def main(argv=None):
         return run_kernel_case(args)
     if args.sweep:
         return run_sweep(args)
+    if args.workload == "dense8b":
+        return run_dense8b(args)
     return run_ours(args)
 
 

@@ -85,10 +85,20 @@ enum {
     NVFP4_COLWISE = 2,    /* produce out_col: x^T quantized along x's rows (K = rows)    */
     NVFP4_BLOCK2D = 4,    /* one scale per 16x16 tile (weights); RTN only                */
     NVFP4_SR = 8,         /* stochastic rounding (gradients)                             */
-    NVFP4_AMAX_GIVEN = 16 /* skip the amax pass: read the tensor amax from the output
+    NVFP4_AMAX_GIVEN = 16,/* skip the amax pass: read the tensor amax from the output
                              operand's `amax` (out_row's if present, else out_col's); the
                              data must then be finite                                    */
+    NVFP4_MX = 32         /* MXFP4 instead of NVFP4 (see below); not with NVFP4_BLOCK2D  */
 };
+
+/* MXFP4, the comparison format of [P1 Formato NVFP4; Nuevo Formato NVFP4] (OCP MX):
+ * E2M1 codes in blocks of 32 along K sharing one power-of-two scale X = 2^E, E =
+ * floor(log2 b) - 2 for the block's largest magnitude b (clamped to [-127, 127]; -127 for a
+ * zero block), stored as the E8M0 byte E + 127; elements E2M1(v / X) rounded to nearest even
+ * (or stochastically with NVFP4_SR), saturating at 6; no tensor scale.  An MXFP4 operand has
+ * the NVFP4 operand's layout: each 32-block's E8M0 byte fills both of its 16-element scale
+ * slots, and `amax` holds the tensor amax only to flag non-finite data.  Multiply MXFP4
+ * operands with nvfp4_gemm_mx. */
 
 /* GEMM output types. */
 enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 };
@@ -169,8 +179,8 @@ nvfp4_status nvfp4_quantize(const void* x_bf16, int64_t rows, int64_t cols, int6
  * transformed (y = (1/4) H diag(s) x), then quantized along the same axis in 1x16 blocks.
  * The amax is that of the transformed tensor.
  *   sign_mask: bit i set = sign -1 for element i of each 16-block.
- *   flags    : NVFP4_SR and/or NVFP4_AMAX_GIVEN (NVFP4_COLWISE is implied; other bits are
- *              rejected).
+ *   flags    : NVFP4_SR, NVFP4_AMAX_GIVEN and/or NVFP4_MX (NVFP4_COLWISE is implied; other
+ *              bits are rejected).
  *   out_col  : cols x rows operand (K = rows).
  * Shape rules: rows a multiple of 64, cols a multiple of 16, ld >= cols, ld % 8 == 0.
  */
@@ -201,6 +211,14 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
                                     uint64_t offset, const nvfp4_operand* out_row,
                                     const nvfp4_operand* out_col, void* workspace,
                                     int* dev_status, void* stream);
+
+/*
+ * nvfp4_gemm for two MXFP4 operands (quantized with NVFP4_MX): the same tensor-core GEMM
+ * with E8M0 block scales and no tensor scales, D = A . B^T.  Arguments, shape rules and
+ * errors as nvfp4_gemm.
+ */
+nvfp4_status nvfp4_gemm_mx(const nvfp4_operand* A, const nvfp4_operand* B, void* D, int d_dtype,
+                           int64_t ldd, int* dev_status, void* stream);
 
 /*
  * Block-scaled FP4 GEMM on the tcgen05 tensor cores: D = A . B^T.

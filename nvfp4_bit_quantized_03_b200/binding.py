@@ -17,7 +17,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "nvfp4.h")
 # status codes and flags (include/nvfp4.h)
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_DEVICE, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_ARG = range(9)
 DEVSTAT_NONFINITE, DEVSTAT_TIMEOUT = 1, 2
-ROWWISE, COLWISE, BLOCK2D, SR, AMAX_GIVEN = 1, 2, 4, 8, 16
+ROWWISE, COLWISE, BLOCK2D, SR, AMAX_GIVEN, MX = 1, 2, 4, 8, 16, 32
 OUT_F32, OUT_BF16 = 0, 1
 
 
@@ -68,6 +68,8 @@ def lib():
         L.nvfp4_quantize_row_rht.restype = i32
         L.nvfp4_gemm.argtypes = [op, op, vp, i32, i64, vp, vp]
         L.nvfp4_gemm.restype = i32
+        L.nvfp4_gemm_mx.argtypes = [op, op, vp, i32, i64, vp, vp]
+        L.nvfp4_gemm_mx.restype = i32
         L.nvfp4_linear_fprop.argtypes = [vp, vp, i64, i64, i64, vp, i32, vp, vp, vp]
         L.nvfp4_linear_fprop.restype = i32
         L.nvfp4_linear_dgrad.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, i32, vp, vp, vp]
@@ -229,17 +231,18 @@ def _check_out(out, rows, cols, what):
                          f"column stride, got {tuple(out.shape)} strides {out.stride()}")
 
 
-def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None):
-    """nvfp4_gemm: D = A . B^T (A, B QuantizedTensor).  The output type is out.dtype when
-    `out` is given, else `out_dtype`."""
+def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None, mx=False):
+    """nvfp4_gemm (nvfp4_gemm_mx with `mx`): D = A . B^T (A, B QuantizedTensor).  The output
+    type is out.dtype when `out` is given, else `out_dtype`."""
+    name = "nvfp4_gemm_mx" if mx else "nvfp4_gemm"
     if out is None:
         out = torch.empty((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
-    _check_out(out, A.rows, B.rows, "nvfp4_gemm")
+    _check_out(out, A.rows, B.rows, name)
     d_dtype = _dtype_code(out.dtype)
     oa, ob = A.operand(), B.operand()
-    st = lib().nvfp4_gemm(ctypes.byref(oa), ctypes.byref(ob), _ptr(out), d_dtype, out.stride(0),
-                          _ptr(dev_status), _stream(stream))
-    _check(st, "nvfp4_gemm")
+    st = getattr(lib(), name)(ctypes.byref(oa), ctypes.byref(ob), _ptr(out), d_dtype,
+                              out.stride(0), _ptr(dev_status), _stream(stream))
+    _check(st, name)
     return out
 
 

@@ -144,12 +144,13 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
 {
     const bool want_row = flags & NVFP4_ROWWISE, want_col = flags & NVFP4_COLWISE;
     const bool b2d = flags & NVFP4_BLOCK2D, sr = flags & NVFP4_SR;
-    const bool given = flags & NVFP4_AMAX_GIVEN;
+    const bool given = flags & NVFP4_AMAX_GIVEN, mx = flags & NVFP4_MX;
     if (flags & ~static_cast<unsigned>(NVFP4_ROWWISE | NVFP4_COLWISE | NVFP4_BLOCK2D | NVFP4_SR |
-                                       NVFP4_AMAX_GIVEN))
+                                       NVFP4_AMAX_GIVEN | NVFP4_MX))
         return NVFP4_ERR_ARG;
     if (!want_row && !want_col) return NVFP4_ERR_ARG;
     if (b2d && sr) return NVFP4_ERR_ARG;
+    if (mx && b2d) return NVFP4_ERR_ARG;
     if (rht && (want_row || b2d)) return NVFP4_ERR_ARG;
     nvfp4_status st = check_input(x, rows, cols, ld, want_row, want_col, out_row, out_col,
                                   given, workspace);
@@ -170,7 +171,7 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
                                    static_cast<uint32_t*>(workspace), grid, s));
         if (st != NVFP4_OK) return st;
     }
-    if (want_row && !want_col && !b2d) {
+    if (want_row && !want_col && !b2d && !mx) {
         return from_cuda(launch_quant_rowwise(
             xs, rows, cols, ld, src, out_row->amax, nullptr, static_cast<uint8_t*>(out_row->codes),
             static_cast<uint8_t*>(out_row->scales), sr, seed, offset, dev_status, sms, s));
@@ -197,7 +198,7 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
     a.offset = offset;
     a.offset_col = offset;
     a.dev_status = dev_status;
-    return from_cuda(launch_quant_tile(a, want_row, want_col, b2d, rht, sr, sms, s));
+    return from_cuda(launch_quant_tile(a, want_row, want_col, b2d, rht, sr, mx, sms, s));
 }
 
 }  // namespace
@@ -290,7 +291,7 @@ nvfp4_status nvfp4_rht_quantize(const void* x_bf16, int64_t rows, int64_t cols, 
                                 uint64_t offset, const nvfp4_operand* out_col,
                                 void* workspace, int* dev_status, void* stream)
 {
-    if (flags & ~static_cast<unsigned>(NVFP4_SR | NVFP4_AMAX_GIVEN | NVFP4_COLWISE))
+    if (flags & ~static_cast<unsigned>(NVFP4_SR | NVFP4_AMAX_GIVEN | NVFP4_COLWISE | NVFP4_MX))
         return NVFP4_ERR_ARG;
     return quantize_impl(x_bf16, rows, cols, ld, flags | NVFP4_COLWISE, true, sign_mask, seed,
                          offset, nullptr, out_col, workspace, dev_status, stream);
@@ -346,11 +347,11 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
     a.offset = offset;
     a.offset_col = offset + 1;
     a.dev_status = dev_status;
-    return from_cuda(launch_quant_tile(a, true, true, false, true, sr, sms, s));
+    return from_cuda(launch_quant_tile(a, true, true, false, true, sr, false, sms, s));
 }
 
-nvfp4_status nvfp4_gemm(const nvfp4_operand* A, const nvfp4_operand* B, void* D, int d_dtype,
-                        int64_t ldd, int* dev_status, void* stream)
+static nvfp4_status gemm_impl(const nvfp4_operand* A, const nvfp4_operand* B, void* D,
+                              int d_dtype, int64_t ldd, int* dev_status, void* stream, bool mx)
 {
     if (!A || !B || !D) return NVFP4_ERR_NULL;
     if (!A->codes || !A->scales || !A->amax || !B->codes || !B->scales || !B->amax)
@@ -382,7 +383,20 @@ nvfp4_status nvfp4_gemm(const nvfp4_operand* A, const nvfp4_operand* B, void* D,
     g.ldd = ldd;
     g.out_bf16 = d_dtype == NVFP4_OUT_BF16;
     g.dev_status = dev_status;
+    g.mx = mx;
     return from_cuda(launch_gemm(g, sms, static_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_gemm(const nvfp4_operand* A, const nvfp4_operand* B, void* D, int d_dtype,
+                        int64_t ldd, int* dev_status, void* stream)
+{
+    return gemm_impl(A, B, D, d_dtype, ldd, dev_status, stream, false);
+}
+
+nvfp4_status nvfp4_gemm_mx(const nvfp4_operand* A, const nvfp4_operand* B, void* D, int d_dtype,
+                           int64_t ldd, int* dev_status, void* stream)
+{
+    return gemm_impl(A, B, D, d_dtype, ldd, dev_status, stream, true);
 }
 
 static nvfp4_status check_linear(const void* p0, const void* p1, void* out, void* workspace,

@@ -92,9 +92,11 @@ constexpr int kDevTimeoutBit = 2;       // NVFP4_DEVSTAT_TIMEOUT
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format 1), both
-// K-major, UE4M3 scales (bit 23 = 0), N >> 3 at bit 17, M >> 4 at bit 24, dense K = 64.
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24, dense K = 64; bit 23 selects the scale type:
+// 0 = UE4M3 (NVFP4), 1 = UE8M0 (MXFP4, whose 32-block scales fill both 16-element slots).
 constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
                            (static_cast<uint32_t>(BM >> 4) << 24);
+constexpr uint32_t IDESC_UE8M0 = IDESC | (1u << 23);
 
 struct Params {
     const uint8_t* sfa;
@@ -240,15 +242,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v)
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+template <bool MX>
 __device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc,
                                          uint32_t sfa, uint32_t sfb, uint32_t accumulate)
 {
+    constexpr uint32_t idesc = MX ? IDESC_UE8M0 : IDESC;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X "
         "[%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
-        "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accumulate), "r"(sfa), "r"(sfb)
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");
 }
 
@@ -351,7 +355,7 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint
     }
 }
 
-template <bool BF16>
+template <bool BF16, bool MX>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
@@ -476,7 +480,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int k = 0; k < nk; ++k) {
                     // K step k = 64 elements = 32 bytes into the 128-byte swizzled rows; its
                     // scales: A in columns tcol + 4k, B in tcol + 16 + 8k
-                    mma_nvf4(tmem_base + ACC_COL, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k),
+                    mma_nvf4<MX>(tmem_base + ACC_COL, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k),
                              tcol + 4 * k, tcol + 16 + 8 * k, (kb | k) != 0 ? 1u : 0u);
                 }
                 any = true;
@@ -557,8 +561,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t stage_buf = smem_u32(staging + (warp - FIRST_EPI_WARP) * STAGING_BYTES);
         const float aa = *p.amax_a, ab = *p.amax_b;
         const bool finite = (aa < INFINITY) && (ab < INFINITY) && aa >= 0.0f && ab >= 0.0f;
+        // NVFP4: undo both tensor scales; MXFP4 has none (its amax only flags bad data)
         const float alpha =
-            finite ? __fdiv_rn(1.0f, __fmul_rn(operand_scale(aa), operand_scale(ab))) : 0.0f;
+            !finite ? 0.0f
+                    : (MX ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(operand_scale(aa), operand_scale(ab))));
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
             // one lane waits, so the whole warp takes the same branch into tcgen05.ld
@@ -657,13 +663,16 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     int dev = 0;
     cudaGetDevice(&dev);
     if (configured_device != dev) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_nvf4_kernel<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             Pipe<true>::SMEM_BYTES);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(gemm_nvf4_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     Pipe<false>::SMEM_BYTES);
+        cudaError_t e = cudaSuccess;
+        const void* kernels[4] = {reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false>),
+                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<false, false>),
+                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<true, true>),
+                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<false, true>)};
+        const int smem[4] = {Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
+                             Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES};
+        for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+            e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     smem[i]);
         if (e != cudaSuccess) return e;
         configured_device = dev;
     }
@@ -685,10 +694,14 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     p.dev_status = g.dev_status;
     const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < sm_count ? tiles : sm_count);
-    if (g.out_bf16)
-        gemm_nvf4_kernel<true><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
+    if (g.out_bf16 && !g.mx)
+        gemm_nvf4_kernel<true, false><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
+    else if (!g.mx)
+        gemm_nvf4_kernel<false, false><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, md, p);
+    else if (g.out_bf16)
+        gemm_nvf4_kernel<true, true><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
     else
-        gemm_nvf4_kernel<false><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, md, p);
+        gemm_nvf4_kernel<false, true><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, md, p);
     return cudaGetLastError();
 }
 

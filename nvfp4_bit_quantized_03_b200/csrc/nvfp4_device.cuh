@@ -157,6 +157,28 @@ __device__ __forceinline__ BlockScale block_scale(float b, float s_enc, const fl
     return out;
 }
 
+// MXFP4 block scale (the pages' comparison format, OCP MX): for a 32-element block whose
+// largest magnitude is b, the shared exponent E = floor(log2 b) - 2 (2 = exponent of E2M1's
+// largest power of two), clamped to [-127, 127] and -127 for b == 0; the scale byte is the
+// E8M0 code E + 127 and the element factor is 2^-E, an exact FP32 power of two (2^-127 is
+// subnormal but representable), so v * 2^-E is one correctly rounded scaling.
+__device__ __forceinline__ BlockScale mx_block_scale(float b)
+{
+    const uint32_t bits = __float_as_uint(b);
+    int fl;                                    // floor(log2 b)
+    if (bits == 0) fl = -200;
+    else if (bits >= 0x00800000u) fl = static_cast<int>(bits >> 23) - 127;
+    else fl = (31 - __clz(static_cast<int>(bits))) - 149;  // subnormal: top set bit
+    int E = fl - 2;
+    E = E < -127 ? -127 : (E > 127 ? 127 : E);
+    BlockScale out;
+    out.sf = static_cast<uint32_t>(E + 127);
+    const int k = -E;
+    out.r = k >= -126 ? __uint_as_float(static_cast<uint32_t>(k + 127) << 23)
+                      : __uint_as_float(0x00400000u);
+    return out;
+}
+
 // ---- E2M1 ------------------------------------------------------------------------------
 
 // Two E2M1 codes (round-to-nearest-even, saturating, sign kept) packed in one byte, the

@@ -68,7 +68,7 @@ cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, 
                                  uint8_t* codes, uint8_t* scales, bool sr, uint64_t seed,
                                  uint64_t offset, int* dev_status, int sm_count, cudaStream_t s);
 cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2d, bool rht,
-                              bool sr, int sm_count, cudaStream_t s);
+                              bool sr, bool mx, int sm_count, cudaStream_t s);
 
 struct GemmArgs {
     const uint8_t* a_codes;
@@ -82,6 +82,7 @@ struct GemmArgs {
     int64_t ldd;
     int out_bf16;
     int* dev_status;
+    bool mx;  // MXFP4 operands: E8M0 scales (each 32-block's byte in both 16-slots), no tensor scale
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s);

@@ -288,7 +288,7 @@ __device__ __forceinline__ void encode16(const float* y, const BlockScale& bs, c
     w1 = p[1];
 }
 
-template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR>
+template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
 __global__ void __launch_bounds__(128, SR ? 6 : 8) quant_tile_kernel(TileArgs a)
 {
     __shared__ __align__(16) uint16_t tile[kTileRows * kTilePitch];
@@ -368,8 +368,26 @@ __global__ void __launch_bounds__(128, SR ? 6 : 8) quant_tile_kernel(TileArgs a)
             const int64_t r = r0 + rrow;
             uint32_t words[8];
             uint32_t sfw = 0;
+            if (MX) {
+                // 32-element blocks: the pairs (0, 1) and (2, 3) of this thread's 16-blocks
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+                for (int pr = 0; pr < 2; ++pr) {
+                    float v0[16], v1[16];
+                    load_row_block(2 * pr, v0);
+                    load_row_block(2 * pr + 1, v1);
+                    float b = 0.0f;
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) b = fmaxf(b, fmaxf(fabsf(v0[j]), fabsf(v1[j])));
+                    const BlockScale bs = mx_block_scale(b);
+                    const uint64_t e0 = static_cast<uint64_t>(r) * a.cols + c0 + (rblk + 2 * pr) * 16;
+                    encode16<SR>(v0, bs, philox, e0, a.offset, words[4 * pr], words[4 * pr + 1]);
+                    encode16<SR>(v1, bs, philox, e0 + 16, a.offset, words[4 * pr + 2],
+                                 words[4 * pr + 3]);
+                    sfw |= (bs.sf | (bs.sf << 8)) << (16 * pr);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < (MX ? 0 : 4); ++q) {
                 float rv[16];
                 load_row_block(q, rv);
                 float b;
@@ -401,8 +419,33 @@ __global__ void __launch_bounds__(128, SR ? 6 : 8) quant_tile_kernel(TileArgs a)
             const int64_t orow = c0 + t;  // output row = input column
             uint32_t words[8];
             uint32_t sfw = 0;
+            auto load_col_block = [&](int q, float* y) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+                for (int i = 0; i < 16; ++i)
+                    y[i] = __uint_as_float(static_cast<uint32_t>(
+                               tile[(q * 16 + i) * kTilePitch + t]) << 16);
+                if (RHT) rht16(y, a.sign_mask);
+            };
+            if (MX) {
+                // 32-element blocks along the rows: the pairs (0, 1) and (2, 3) of 16-blocks
+#pragma unroll
+                for (int pr = 0; pr < 2; ++pr) {
+                    float y0[16], y1[16];
+                    load_col_block(2 * pr, y0);
+                    load_col_block(2 * pr + 1, y1);
+                    float b = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) b = fmaxf(b, fmaxf(fabsf(y0[i]), fabsf(y1[i])));
+                    const BlockScale bs = mx_block_scale(b);
+                    const uint64_t e0 = static_cast<uint64_t>(orow) * a.rows + r0 + pr * 32;
+                    encode16<SR>(y0, bs, philox, e0, a.offset_col, words[4 * pr], words[4 * pr + 1]);
+                    encode16<SR>(y1, bs, philox, e0 + 16, a.offset_col, words[4 * pr + 2],
+                                 words[4 * pr + 3]);
+                    sfw |= (bs.sf | (bs.sf << 8)) << (16 * pr);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < (MX ? 0 : 4); ++q) {
                 float y[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i)
@@ -520,24 +563,39 @@ cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, 
     return cudaGetLastError();
 }
 
-template <bool ROW, bool COL, bool B2D, bool RHT, bool SR>
+template <bool ROW, bool COL, bool B2D, bool RHT, bool SR, bool MX = false>
 static void launch_tile_t(const TileArgs& a, int64_t ntiles, int sm_count, cudaStream_t s)
 {
-    static const int resident = resident_ctas(quant_tile_kernel<ROW, COL, B2D, RHT, SR>, 128);
+    static const int resident =
+        resident_ctas(quant_tile_kernel<ROW, COL, B2D, RHT, SR, MX>, 128);
     int64_t grid = static_cast<int64_t>(sm_count) * resident;
     if (grid > ntiles) grid = ntiles;
     if (grid < 1) grid = 1;
-    quant_tile_kernel<ROW, COL, B2D, RHT, SR><<<static_cast<int>(grid), 128, 0, s>>>(a);
+    quant_tile_kernel<ROW, COL, B2D, RHT, SR, MX><<<static_cast<int>(grid), 128, 0, s>>>(a);
 }
 
 cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2d, bool rht,
-                              bool sr, int sm_count, cudaStream_t s)
+                              bool sr, bool mx, int sm_count, cudaStream_t s)
 {
     const int64_t ntiles = ((a.rows + kTileRows - 1) / kTileRows) *
                            ((a.cols + kTileCols - 1) / kTileCols);
     const int64_t g = ntiles;
     const int sm = sm_count;
     // Supported combinations (the API rejects the others before launching).
+    if (mx) {
+        // MXFP4: row-wise and/or column-wise (the latter optionally RHT'd), RTN or SR
+        if (block2d || (row && rht)) return cudaErrorInvalidValue;
+        if (row && col && sr)        launch_tile_t<true, true, false, false, true, true>(a, g, sm, s);
+        else if (row && col)         launch_tile_t<true, true, false, false, false, true>(a, g, sm, s);
+        else if (row && sr)          launch_tile_t<true, false, false, false, true, true>(a, g, sm, s);
+        else if (row)                launch_tile_t<true, false, false, false, false, true>(a, g, sm, s);
+        else if (col && rht && sr)   launch_tile_t<false, true, false, true, true, true>(a, g, sm, s);
+        else if (col && rht)         launch_tile_t<false, true, false, true, false, true>(a, g, sm, s);
+        else if (col && sr)          launch_tile_t<false, true, false, false, true, true>(a, g, sm, s);
+        else if (col)                launch_tile_t<false, true, false, false, false, true>(a, g, sm, s);
+        else return cudaErrorInvalidValue;
+        return cudaGetLastError();
+    }
     if (row && col && rht && sr)          launch_tile_t<true, true, false, true, true>(a, g, sm, s);
     else if (row && col && rht && !sr)    launch_tile_t<true, true, false, true, false>(a, g, sm, s);
     else if (row && col && block2d)       launch_tile_t<true, true, true, false, false>(a, g, sm, s);

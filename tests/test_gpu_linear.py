@@ -75,12 +75,9 @@ def _sample(n, k=96, seed=0):
     return np.sort(rng.choice(n, size=min(k, n), replace=False))
 
 
-@pytest.mark.slow
-@pytest.mark.parametrize("which", ["up", "down"])
-def test_mlp_12b_sampled(which):
-    """12B-class MLP shapes (tokens 8192, 5120 <-> 20480) in the launch configuration the
-    benchmark times; 96 sampled rows x all columns and all rows x 96 sampled columns."""
-    wl = synth.mlp_12b()
+def _check_workload_linear(wl, which):
+    """fprop, dgrad and wgrad of one linear of a workload through the C ABI against the
+    oracle: 96 sampled rows x all columns and all rows x 96 sampled columns of each GEMM."""
     lin = {l.name: l for l in wl.linears}[which]
     idx = [l.name for l in wl.linears].index(which)
     X, W, dY = synth.linear_inputs(lin, wl.seed, layer_index=idx)
@@ -100,3 +97,19 @@ def test_mlp_12b_sampled(which):
         Dc, nc = oracle.gemm_ref(qa, qb, cols=c)
         assert_gemm_close(D[:, torch.from_numpy(c).cuda()].cpu().numpy(), Dc, nc,
                           what=name + " cols")
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("which", ["up", "down"])
+def test_mlp_12b_sampled(which):
+    """12B-class MLP shapes (tokens 8192, 5120 <-> 20480), the shapes the benchmark times."""
+    _check_workload_linear(synth.mlp_12b(), which)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("which", ["qkv", "o", "down"])
+def test_dense_8b_layer_sampled(which):
+    """8B-class dense layer at tokens 16384, d 4096: QKV 4096 -> 6144, O 4096 -> 4096 and the
+    MLP down-projection 14336 -> 4096 (gate and up share the down-projection's sizes
+    transposed, which the 12B-class case already covers at other sizes)."""
+    _check_workload_linear(synth.dense_8b_layer(), which)
