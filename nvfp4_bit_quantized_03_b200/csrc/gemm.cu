@@ -62,14 +62,14 @@ constexpr int SF_COL = BN;              // scales: 48 columns per stage from col
 constexpr int SF_COLS_PER_STAGE = (BK / MMA_K) * (4 + 8);
 constexpr int BAR_BYTES = 256;
 
-// Pipeline shape per output type.  A bf16 tile (64 KB of output) goes out through 512-byte
-// staging buffers, which leaves room for a fourth operand stage; an FP32 tile (128 KB) keeps
-// 2 KB buffers and three stages.  The epilogue's TMA stores are paced (a first-round delay and
-// a gap between rounds) so that they do not crowd the next tile's first operand loads.
+// Pipeline shape per output type.  Four operand stages either way: a bf16 tile (64 KB of
+// output) goes out through 512-byte staging buffers with paced TMA stores (a first-round delay
+// and a gap between rounds, so that they do not crowd the next tile's first operand loads); an
+// FP32 tile (128 KB) is stored straight from registers (store_f32_direct).
 template <bool BF16>
 struct Pipe {
-    static constexpr int STAGES = BF16 ? 4 : 3;
-    static constexpr int STAGING_BYTES = BF16 ? 512 : 2048;  // per epilogue warp
+    static constexpr int STAGES = 4;
+    static constexpr int STAGING_BYTES = 512;  // per epilogue warp (bf16 boxes; FP32 stores direct)
     static constexpr int SMEM_BYTES =
         STAGES * STAGE_BYTES + NUM_EPI_WARPS * STAGING_BYTES + BAR_BYTES + 1024;
     static constexpr unsigned FIRST_NS = BF16 ? 3000u : 0u;
@@ -278,6 +278,24 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v)
           "=r"(v[31])
         : "r"(taddr));
 }
+// 16 TMEM lanes x 8 groups of 8 FP32 columns: thread t receives, for group g, registers
+// v[4g], v[4g+1] = lane t / 4, columns 8g + 2 (t % 4) + {0, 1}, and v[4g+2], v[4g+3] = the
+// same columns of lane t / 4 + 8 (the 16x256b pattern, repeated 8 times along the columns).
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t* v)
+{
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
+        "[%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr));
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Tensor encode scale of an operand, as the quantizer computed it; see alpha below.
@@ -352,6 +370,33 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint
         __syncwarp();
         const int x = n0 + r * COLS;
         if (lane == 0 && y < M && x < N) tma_store_2d(tmap_d, stage_buf, x, y);
+    }
+}
+
+// One epilogue warp's 32 x 64 FP32 slice straight from registers (the 16x256b layout of
+// tmem_ld_16x256b_x8 for the two 16-row halves): scaled by alpha, each instruction writes 8 B
+// per thread, i.e. 8 rows x 32 contiguous bytes (whole sectors) per warp; no staging, so the
+// FP32 kernel keeps the shared memory for operand stages like the bf16 one.
+__device__ __forceinline__ void store_f32_direct(const uint32_t* v, float alpha, float* D,
+                                                 int64_t ldd, int lane, int n0, int y, int M,
+                                                 int N)
+{
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            const int col = n0 + 8 * g + 2 * (lane & 3);
+            const uint32_t* r = v + 32 * h + 4 * g;
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const int row = y + 16 * h + (lane >> 2) + 8 * k;
+                if (row < M && col < N) {
+                    const float2 val = make_float2(__fmul_rn(__uint_as_float(r[2 * k]), alpha),
+                                                   __fmul_rn(__uint_as_float(r[2 * k + 1]), alpha));
+                    *reinterpret_cast<float2*>(D + static_cast<int64_t>(row) * ldd + col) = val;
+                }
+            }
+        }
     }
 }
 
@@ -578,8 +623,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t v[64];
             const uint32_t taddr = tmem_base + ACC_COL + (static_cast<uint32_t>(32 * q) << 16) +
                                    64 * chunk;
-            tmem_ld32(taddr, v);
-            tmem_ld32(taddr + 32, v + 32);
+            if (BF16) {
+                tmem_ld32(taddr, v);
+                tmem_ld32(taddr + 32, v + 32);
+            } else {
+                // two 16-lane halves; v[32h + 4g ..] = rows (lane / 4, lane / 4 + 8) of the
+                // half, columns 8g + 2 (lane % 4) and the next one
+                tmem_ld_16x256b_x8(taddr, v);
+                tmem_ld_16x256b_x8(taddr + (16u << 16), v + 32);
+            }
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
@@ -589,7 +641,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             tile_coords(t, tiles_m, tiles_n, tm, tn);
             const int y = tm * BM + 32 * q;       // first output row of this warp's slice
             const int n0 = tn * BN + 64 * chunk;  // first output column
-            store_slice<BF16>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
+            if (BF16)
+                store_slice<BF16>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
+            else
+                store_f32_direct(v, alpha, static_cast<float*>(p.D), p.ldd, lane, n0, y, p.M, p.N);
         }
         if (lane == 0) bulk_wait_all();
     }
