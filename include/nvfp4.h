@@ -213,6 +213,15 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
                                     int* dev_status, void* stream);
 
 /*
+ * Self-test of the device-side bounded waits (no counterpart on the pages): queues one kernel
+ * whose thread waits, with the GEMM's own wait routine, on an mbarrier that nothing completes.
+ * After 50 ms the wait gives up, NVFP4_DEVSTAT_TIMEOUT is OR-ed into *dev_status (device,
+ * 4-byte aligned) and the kernel returns; the context stays usable.  This is how the GEMM's
+ * waits end if a copy or an MMA never signals, without hanging the GPU.
+ */
+nvfp4_status nvfp4_selftest_wait_timeout(int* dev_status, void* stream);
+
+/*
  * nvfp4_gemm for two MXFP4 operands (quantized with NVFP4_MX): the same tensor-core GEMM
  * with E8M0 block scales and no tensor scales, D = A . B^T.  Arguments, shape rules and
  * errors as nvfp4_gemm.

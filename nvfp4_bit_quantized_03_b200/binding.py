@@ -70,6 +70,8 @@ def lib():
         L.nvfp4_gemm.restype = i32
         L.nvfp4_gemm_mx.argtypes = [op, op, vp, i32, i64, vp, vp]
         L.nvfp4_gemm_mx.restype = i32
+        L.nvfp4_selftest_wait_timeout.argtypes = [vp, vp]
+        L.nvfp4_selftest_wait_timeout.restype = i32
         L.nvfp4_linear_fprop.argtypes = [vp, vp, i64, i64, i64, vp, i32, vp, vp, vp]
         L.nvfp4_linear_fprop.restype = i32
         L.nvfp4_linear_dgrad.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, i32, vp, vp, vp]
@@ -246,6 +248,13 @@ def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None, 
     return out
 
 
+
+
+def selftest_wait_timeout(dev_status, stream=None):
+    """nvfp4_selftest_wait_timeout: a bounded wait that nothing satisfies; after it the device
+    status word has NVFP4_DEVSTAT_TIMEOUT set."""
+    _check(lib().nvfp4_selftest_wait_timeout(_ptr(dev_status), _stream(stream)),
+           "nvfp4_selftest_wait_timeout")
 
 
 def linear_fprop(X, W, out=None, out_dtype=torch.float32, workspace=None, dev_status=None,

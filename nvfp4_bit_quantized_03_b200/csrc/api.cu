@@ -393,6 +393,17 @@ nvfp4_status nvfp4_gemm(const nvfp4_operand* A, const nvfp4_operand* B, void* D,
     return gemm_impl(A, B, D, d_dtype, ldd, dev_status, stream, false);
 }
 
+nvfp4_status nvfp4_selftest_wait_timeout(int* dev_status, void* stream)
+{
+    if (!dev_status) return NVFP4_ERR_NULL;
+    if (!aligned4(dev_status)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    const nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(launch_wait_selftest(dev_status, 50000000ull,  // 50 ms
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_gemm_mx(const nvfp4_operand* A, const nvfp4_operand* B, void* D, int d_dtype,
                            int64_t ldd, int* dev_status, void* stream)
 {

@@ -152,7 +152,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 // Wait for the phase of `bar` with the given parity to complete.  Gives up when another
 // role has aborted (unless `ignore_abort`) or after WAIT_LIMIT_NS, which it reports.
 __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* dev_status, bool ignore_abort = false)
+                                          int* dev_status, bool ignore_abort = false,
+                                          unsigned long long limit_ns = WAIT_LIMIT_NS)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
@@ -160,7 +161,7 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 31u) == 0) {
             if (!ignore_abort && *abort_flag) return false;
-            if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+            if (globaltimer() - t0 > limit_ns) {
                 *abort_flag = 1;
                 if (dev_status) atomicOr(dev_status, kDevTimeoutBit);
                 return false;
@@ -660,6 +661,20 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 }
 
+// Self-test of the bounded waits: one thread waits on an mbarrier that nothing arrives at, with
+// the GEMM's own wait routine and a limit of `limit_ns`; the wait gives up, records
+// NVFP4_DEVSTAT_TIMEOUT and the kernel returns.
+__global__ void wait_selftest_kernel(int* dev_status, unsigned long long limit_ns)
+{
+    __shared__ __align__(8) uint64_t never;
+    __shared__ int abort_flag;
+    if (threadIdx.x != 0) return;
+    mbar_init(smem_u32(&never), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    wait_bounded(smem_u32(&never), 0, &abort_flag, dev_status, false, limit_ns);
+}
+
 // ---- host side ---------------------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
@@ -712,12 +727,23 @@ bool make_output_map(CUtensorMap* map, void* D, int64_t M, int64_t N, int64_t ld
 
 }  // namespace
 
+cudaError_t launch_wait_selftest(int* dev_status, unsigned long long limit_ns, cudaStream_t s)
+{
+    wait_selftest_kernel<<<1, 32, 0, s>>>(dev_status, limit_ns);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
 {
-    static int configured_device = -1;
+    // the kernels' shared-memory limit is raised once per device
+    constexpr int kDevices = 64;
+    static bool configured[kDevices] = {};
+    static std::mutex configure_mutex;
     int dev = 0;
-    cudaGetDevice(&dev);
-    if (configured_device != dev) {
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices)
+        return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(configure_mutex);
+    if (!configured[dev]) {
         cudaError_t e = cudaSuccess;
         const void* kernels[4] = {reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false>),
                                   reinterpret_cast<const void*>(gemm_nvf4_kernel<false, false>),
@@ -729,7 +755,7 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
             e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      smem[i]);
         if (e != cudaSuccess) return e;
-        configured_device = dev;
+        configured[dev] = true;
     }
     CUtensorMap ma, mb, md;
     if (!make_codes_map(&ma, g.a_codes, g.M, g.K, BM) || !make_codes_map(&mb, g.b_codes, g.N, g.K, BN) ||

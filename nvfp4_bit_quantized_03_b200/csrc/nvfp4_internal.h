@@ -86,5 +86,8 @@ struct GemmArgs {
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s);
+// A kernel whose only thread waits, with the GEMM's bounded-wait routine, on an mbarrier that
+// nothing completes; it records NVFP4_DEVSTAT_TIMEOUT after limit_ns and returns.
+cudaError_t launch_wait_selftest(int* dev_status, unsigned long long limit_ns, cudaStream_t s);
 
 }  // namespace nvfp4

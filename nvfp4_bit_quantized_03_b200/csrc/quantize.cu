@@ -65,6 +65,12 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
                                                        uint32_t* __restrict__ partials,
                                                        uint32_t* __restrict__ partials_plain)
 {
+    // The transform's sign flips are applied to the packed bf16 pairs (one xor per two
+    // values), and its final x1/4 is applied once to the maximum: rounding is monotone, so the
+    // largest |RN(v / 4)| is RN(max |v| / 4) -- the same bits as transforming exactly.
+    uint32_t flip[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) flip[k] = ((sign_mask >> k) & 1u) ? 0x80008000u : 0u;
     uint32_t mp = 0;
     const int64_t cpr = cols >> 2;  // 8-byte column groups per row
     const int64_t total = (rows >> 4) * cpr;
@@ -87,14 +93,25 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
             float y[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const uint32_t w = j < 2 ? v[k].x : v[k].y;
+                const uint32_t w = (j < 2 ? v[k].x : v[k].y) ^ flip[k];
                 y[k] = (j & 1) ? bf16_hi(w) : bf16_lo(w);
             }
-            rht16(y, sign_mask);
 #pragma unroll
-            for (int k = 0; k < 16; ++k) m = max(m, __float_as_uint(fabsf(y[k])));
+            for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    if (k & h) continue;
+                    const float a = y[k], b = y[k + h];
+                    y[k] = __fadd_rn(a, b);
+                    y[k + h] = __fsub_rn(a, b);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) m = max(m, __float_as_uint(y[k]) & 0x7FFFFFFFu);
         }
     }
+    // x1/4 of the largest magnitude (NaN and Inf stay at or above the Inf pattern)
+    m = __float_as_uint(__fmul_rn(__uint_as_float(m), 0.25f));
     block_max_store(m, partials + blockIdx.x);
     if (PLAIN) {
         __syncthreads();  // block_max_store's shared scratch is reused

@@ -186,3 +186,8 @@ def test_binding_rejects_bad_output_tensors_before_calling():
         B.gemm(A, Bq, out=torch.empty((128, 200), dtype=torch.float32))
     with pytest.raises(ValueError):  # host tensor
         B.gemm(A, Bq, out=torch.empty((128, 256), dtype=torch.bfloat16))
+
+
+def test_wait_selftest_rejects_a_null_status_word():
+    # argument checks come before any device access
+    assert B.lib().nvfp4_selftest_wait_timeout(None, None) == B.ERR_NULL
