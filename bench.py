@@ -482,15 +482,34 @@ def run_kernel_case(args):
     T, D, F = 8192, 5120, 20480
     dev = torch.device("cuda", torch.cuda.current_device())
     ws = torch.empty((B.workspace_bytes(1 << 14, 1 << 14),), dtype=torch.uint8, device=dev)
-    if args.kernel == "gemm":
+    if args.kernel in ("gemm", "gemm_amax", "chain", "chain_amax"):
         X = torch.from_numpy(synth.activations((T, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
         W = torch.from_numpy(synth.weights((F, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
         qa, _ = B.quantize(X, B.ROWWISE, workspace=ws)
         qb, _ = B.quantize(W, B.ROWWISE | B.BLOCK2D, workspace=ws)
         out = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
-        fn = lambda: B.gemm(qa, qb, out=out)  # noqa: E731
+        amax = torch.empty(2, dtype=torch.float32, device=dev)
+        qr, qc = B.QuantizedTensor(T, F, dev), B.QuantizedTensor(F, T, dev)
+
+        def chain():
+            # the GEMM output quantized for the next layer: row-wise and RHT'd column-wise, SR
+            B.gemm(qa, qb, out=out)
+            B.quantize_row_rht(out, 0x5A3C, B.SR, seed=1, out_row=qr, out_col=qc, workspace=ws)
+
+        def chain_amax():
+            # the same, with both maxima taken in the GEMM's epilogue instead of an amax pass;
+            # the two quantized outputs read them in place
+            qr.amax, qc.amax = amax[0:1], amax[1:2]
+            B.gemm_amax(qa, qb, 0x5A3C, out=out, amax_out=amax)
+            B.quantize_row_rht(out, 0x5A3C, B.SR | B.AMAX_GIVEN, seed=1, out_row=qr,
+                               out_col=qc)
+
+        fn = {"gemm": lambda: B.gemm(qa, qb, out=out),
+              "gemm_amax": lambda: B.gemm_amax(qa, qb, 0x5A3C, out=out, amax_out=amax),
+              "chain": chain, "chain_amax": chain_amax}[args.kernel]
         work, unit, peak = 2 * T * D * F / 1e12, "TFLOP/s", peaks["bf16_tflops"] * FP4_OVER_BF16
-        shape = f"M={T} N={F} K={D}, bf16 out"
+        shape = f"M={T} N={F} K={D}, bf16 out" + (
+            ", then SR dual quantization of D" if args.kernel.startswith("chain") else "")
     else:
         x = torch.from_numpy(synth.gradients((T, F), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
         n = T * F
@@ -681,7 +700,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["gemm", "rowwise", "tile2d", "rht", "dual"], default=None,
+    ap.add_argument("--kernel", choices=["gemm", "gemm_amax", "chain", "chain_amax", "rowwise",
+                                         "tile2d", "rht", "dual"], default=None,
                     help="time one kernel family alone at the workload's shapes (profiling)")
     ap.add_argument("--sweep", action="store_true",
                     help="quantizer bandwidth sweep over 2^n-element tensors (one line per point)")

@@ -213,6 +213,23 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
                                     int* dev_status, void* stream);
 
 /*
+ * nvfp4_gemm with bf16 output that also emits the two maxima the next quantization of D needs.
+ * The recipe's tensor scales come from the amax of the quantized tensor [P1 Formato NVFP4],
+ * and a layer's output D is the next layer's input (or, from dgrad, the previous layer's
+ * output gradient), quantized row-wise and RHT'd column-wise [P1 RHT].
+ *   amax_out : device, 2 FP32 (4-byte aligned), overwritten: amax_out[0] = max |D| and
+ *              amax_out[1] = max |RHT(D)| (16x16 transform of every 16 consecutive rows of each
+ *              column with sign_mask), both over D as stored in bf16 -- exactly the amax values
+ *              nvfp4_quantize_row_rht(D, sign_mask) computes.  NaN or Inf in D gives a value
+ *              at or above +Inf.
+ * Pass them to nvfp4_quantize_row_rht with NVFP4_AMAX_GIVEN (out_row->amax = &amax_out[0],
+ * out_col->amax = &amax_out[1]) to skip its amax pass.  Other arguments as nvfp4_gemm.
+ */
+nvfp4_status nvfp4_gemm_amax(const nvfp4_operand* A, const nvfp4_operand* B, void* D_bf16,
+                             int64_t ldd, uint16_t sign_mask, float* amax_out, int* dev_status,
+                             void* stream);
+
+/*
  * Self-test of the device-side bounded waits (no counterpart on the pages): queues one kernel
  * whose thread waits, with the GEMM's own wait routine, on an mbarrier that nothing completes.
  * After 50 ms the wait gives up, NVFP4_DEVSTAT_TIMEOUT is OR-ed into *dev_status (device,

@@ -70,6 +70,8 @@ def lib():
         L.nvfp4_gemm.restype = i32
         L.nvfp4_gemm_mx.argtypes = [op, op, vp, i32, i64, vp, vp]
         L.nvfp4_gemm_mx.restype = i32
+        L.nvfp4_gemm_amax.argtypes = [op, op, vp, i64, u16, vp, vp, vp]
+        L.nvfp4_gemm_amax.restype = i32
         L.nvfp4_selftest_wait_timeout.argtypes = [vp, vp]
         L.nvfp4_selftest_wait_timeout.restype = i32
         L.nvfp4_linear_fprop.argtypes = [vp, vp, i64, i64, i64, vp, i32, vp, vp, vp]
@@ -248,6 +250,19 @@ def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None, 
     return out
 
 
+def gemm_amax(A, B, sign_mask, out=None, amax_out=None, dev_status=None, stream=None):
+    """nvfp4_gemm_amax: bf16 D = A . B^T plus amax_out = [max |D|, max |RHT(D)|] (FP32)."""
+    if out is None:
+        out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
+    _check_out(out, A.rows, B.rows, "nvfp4_gemm_amax")
+    assert out.dtype == torch.bfloat16
+    if amax_out is None:
+        amax_out = torch.empty(2, dtype=torch.float32, device=A.codes.device)
+    oa, ob = A.operand(), B.operand()
+    st = lib().nvfp4_gemm_amax(ctypes.byref(oa), ctypes.byref(ob), _ptr(out), out.stride(0),
+                               sign_mask, _ptr(amax_out), _ptr(dev_status), _stream(stream))
+    _check(st, "nvfp4_gemm_amax")
+    return out, amax_out
 
 
 def selftest_wait_timeout(dev_status, stream=None):

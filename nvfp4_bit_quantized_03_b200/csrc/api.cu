@@ -351,7 +351,8 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
 }
 
 static nvfp4_status gemm_impl(const nvfp4_operand* A, const nvfp4_operand* B, void* D,
-                              int d_dtype, int64_t ldd, int* dev_status, void* stream, bool mx)
+                              int d_dtype, int64_t ldd, int* dev_status, void* stream, bool mx,
+                              float* amax_out = nullptr, uint32_t sign_mask = 0)
 {
     if (!A || !B || !D) return NVFP4_ERR_NULL;
     if (!A->codes || !A->scales || !A->amax || !B->codes || !B->scales || !B->amax)
@@ -384,6 +385,8 @@ static nvfp4_status gemm_impl(const nvfp4_operand* A, const nvfp4_operand* B, vo
     g.out_bf16 = d_dtype == NVFP4_OUT_BF16;
     g.dev_status = dev_status;
     g.mx = mx;
+    g.amax_out = reinterpret_cast<uint32_t*>(amax_out);
+    g.sign_mask = sign_mask;
     return from_cuda(launch_gemm(g, sms, static_cast<cudaStream_t>(stream)));
 }
 
@@ -408,6 +411,16 @@ nvfp4_status nvfp4_gemm_mx(const nvfp4_operand* A, const nvfp4_operand* B, void*
                            int64_t ldd, int* dev_status, void* stream)
 {
     return gemm_impl(A, B, D, d_dtype, ldd, dev_status, stream, true);
+}
+
+nvfp4_status nvfp4_gemm_amax(const nvfp4_operand* A, const nvfp4_operand* B, void* D_bf16,
+                             int64_t ldd, uint16_t sign_mask, float* amax_out, int* dev_status,
+                             void* stream)
+{
+    if (!amax_out) return NVFP4_ERR_NULL;
+    if (!aligned4(amax_out)) return NVFP4_ERR_ALIGN;
+    return gemm_impl(A, B, D_bf16, NVFP4_OUT_BF16, ldd, dev_status, stream, false, amax_out,
+                     sign_mask);
 }
 
 static nvfp4_status check_linear(const void* p0, const void* p1, void* out, void* workspace,

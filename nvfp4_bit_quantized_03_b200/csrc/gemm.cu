@@ -99,6 +99,8 @@ constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >>
 constexpr uint32_t IDESC_UE8M0 = IDESC | (1u << 23);
 
 struct Params {
+    uint32_t* amax_out;  // fused maxima (bf16 output only): [max |D|, max |RHT(D)|] as FP32 bits
+    uint32_t sign_mask;  // RHT signs for amax_out[1]
     const uint8_t* sfa;
     const uint8_t* sfb;
     const float* amax_a;
@@ -330,10 +332,18 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 //    c ^ ((row / 2) % 4)), which the tensor map undoes.
 // Each round waits only for the previous box to leave the buffer; rounds are paced by
 // Pipe::FIRST_NS / GAP_NS.
-template <bool BF16>
+// With AMAX (bf16 only) the warp also folds its slice into the two maxima the next quantizer
+// of D needs: m_plain, the largest |bf16| bit pattern (in the low 16 bits of each half), and
+// m_rht, the largest |v| bit pattern of the random Hadamard transform of every 16 consecutive
+// rows (lanes 0-15 and 16-31; lane = row) before its x1/4: the sign of row i flips when bit i of
+// sign_mask is set, then butterflies of widths 1, 2, 4, 8 across lanes (shfl_xor), the lower
+// lane keeping a + b and the upper a - b -- the same FP32 operations, in the same order, as the
+// quantizer's transform of the bf16 values.
+template <bool BF16, bool AMAX = false>
 __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint32_t stage_buf,
                                             int lane, const CUtensorMap* tmap_d, int n0, int y,
-                                            int M, int N)
+                                            int M, int N, uint32_t* m_plain = nullptr,
+                                            uint32_t* m_rht = nullptr, uint32_t flip = 0)
 {
     using P = Pipe<BF16>;
     constexpr int CHUNKS = BF16 ? 1 : 4;             // 16-byte chunks per box row
@@ -357,6 +367,27 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint
                         __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j]), alpha),
                                               __fmul_rn(__uint_as_float(v[j + 1]), alpha));
                     o[h] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+                if (AMAX) {
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) *m_plain = __vmaxu2(*m_plain, o[h] & 0x7FFF7FFFu);
+                    float f[8];
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        f[2 * h] = __uint_as_float((o[h] << 16) ^ flip);
+                        f[2 * h + 1] = __uint_as_float((o[h] & 0xFFFF0000u) ^ flip);
+                    }
+#pragma unroll
+                    for (int w = 1; w < 16; w <<= 1) {
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const float other = __shfl_xor_sync(0xFFFFFFFFu, f[k], w);
+                            f[k] = (lane & w) ? __fsub_rn(other, f[k]) : __fadd_rn(f[k], other);
+                        }
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        *m_rht = max(*m_rht, __float_as_uint(f[k]) & 0x7FFFFFFFu);
                 }
             } else {
 #pragma unroll
@@ -401,7 +432,7 @@ __device__ __forceinline__ void store_f32_direct(const uint32_t* v, float alpha,
     }
 }
 
-template <bool BF16, bool MX>
+template <bool BF16, bool MX, bool AMAX = false>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
@@ -612,6 +643,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             !finite ? 0.0f
                     : (MX ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(operand_scale(aa), operand_scale(ab))));
         int it = 0;
+        uint32_t m_plain = 0, m_rht = 0;  // fused maxima (AMAX)
+        const uint32_t flip = ((p.sign_mask >> (lane & 15)) & 1u) ? 0x80000000u : 0u;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
             // one lane waits, so the whole warp takes the same branch into tcgen05.ld
             bool ready = lane == 0 ? wait_bounded(bar(BAR_ACC_FULL), it & 1, abort_flag,
@@ -643,11 +676,21 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int y = tm * BM + 32 * q;       // first output row of this warp's slice
             const int n0 = tn * BN + 64 * chunk;  // first output column
             if (BF16)
-                store_slice<BF16>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N);
+                store_slice<BF16, AMAX>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N,
+                                        &m_plain, &m_rht, flip);
             else
                 store_f32_direct(v, alpha, static_cast<float*>(p.D), p.ldd, lane, n0, y, p.M, p.N);
         }
         if (lane == 0) bulk_wait_all();
+        if (AMAX) {
+            m_plain = __reduce_max_sync(0xFFFFFFFFu, max(m_plain & 0xFFFFu, m_plain >> 16) << 16);
+            m_rht = __reduce_max_sync(0xFFFFFFFFu, m_rht);
+            if (lane == 0) {
+                atomicMax(p.amax_out, m_plain);
+                // x1/4 once, on the maximum (rounding is monotone)
+                atomicMax(p.amax_out + 1, __float_as_uint(__fmul_rn(__uint_as_float(m_rht), 0.25f)));
+            }
+        }
     }
 
     tc_fence_before();
@@ -745,13 +788,15 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     std::lock_guard<std::mutex> lock(configure_mutex);
     if (!configured[dev]) {
         cudaError_t e = cudaSuccess;
-        const void* kernels[4] = {reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false>),
+        const void* kernels[5] = {reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false>),
                                   reinterpret_cast<const void*>(gemm_nvf4_kernel<false, false>),
                                   reinterpret_cast<const void*>(gemm_nvf4_kernel<true, true>),
-                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<false, true>)};
-        const int smem[4] = {Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
-                             Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES};
-        for (int i = 0; i < 4 && e == cudaSuccess; ++i)
+                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<false, true>),
+                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false, true>)};
+        const int smem[5] = {Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
+                             Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
+                             Pipe<true>::SMEM_BYTES};
+        for (int i = 0; i < 5 && e == cudaSuccess; ++i)
             e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      smem[i]);
         if (e != cudaSuccess) return e;
@@ -773,9 +818,18 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     p.K = static_cast<int>(g.K);
     p.out_bf16 = g.out_bf16;
     p.dev_status = g.dev_status;
+    p.amax_out = g.amax_out;
+    p.sign_mask = g.sign_mask;
     const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < sm_count ? tiles : sm_count);
-    if (g.out_bf16 && !g.mx)
+    if (g.amax_out) {
+        // fused maxima of the bf16 output for the next quantizer (the API allows it only there)
+        if (!g.out_bf16 || g.mx) return cudaErrorInvalidValue;
+        const cudaError_t e = cudaMemsetAsync(g.amax_out, 0, 2 * sizeof(uint32_t), s);
+        if (e != cudaSuccess) return e;
+        gemm_nvf4_kernel<true, false, true>
+            <<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
+    } else if (g.out_bf16 && !g.mx)
         gemm_nvf4_kernel<true, false><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
     else if (!g.mx)
         gemm_nvf4_kernel<false, false><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, md, p);

@@ -83,6 +83,8 @@ struct GemmArgs {
     int out_bf16;
     int* dev_status;
     bool mx;  // MXFP4 operands: E8M0 scales (each 32-block's byte in both 16-slots), no tensor scale
+    uint32_t* amax_out;  // non-null: fused [max |D|, max |RHT(D)|] (FP32 bits) of a bf16 D
+    uint32_t sign_mask;  // RHT signs for amax_out[1]
 };
 
 cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s);

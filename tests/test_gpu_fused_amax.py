@@ -1,0 +1,80 @@
+"""nvfp4_gemm_amax: a bf16 GEMM that also emits the maxima the next quantization of its output
+needs (max |D| and max |RHT(D)| along the rows), so that quantization can skip its amax pass.
+
+D is a GPU result, so no oracle value is derived from it; the checks are properties that hold
+at any size:
+* D is bit-identical to nvfp4_gemm's bf16 output and matches the oracle's FP64 product within
+  the usual tolerance;
+* the fused maxima equal, bit for bit, the ones the quantizer's own amax pass computes on D;
+* quantizing D with the fused maxima (NVFP4_AMAX_GIVEN) gives exactly the codes, scales and
+  amax of the quantization that runs its amax pass."""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from nvfp4_testlib import assert_gemm_close, need_gpu, to_device_bf16
+
+nv = pytest.importorskip("nvfp4_bit_quantized_03_b200")
+B = nv.binding
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    need_gpu()
+
+
+def _operands(M, N, K, seed):
+    X = synth.activations((M, K), seed=seed)
+    W = synth.weights((N, K), seed=seed)
+    qa, _ = B.quantize(to_device_bf16(X), B.ROWWISE)
+    qb, _ = B.quantize(to_device_bf16(W), B.ROWWISE | B.BLOCK2D)
+    return X, W, qa, qb
+
+
+@pytest.mark.parametrize("M,N,K", [(256, 512, 512), (192, 320, 320), (1024, 2048, 1024)])
+def test_fused_maxima_equal_the_quantizers_amax(M, N, K):
+    X, W, qa, qb = _operands(M, N, K, seed=50)
+    mask = oracle.sign_mask_from_seed(50)
+    D, amax = B.gemm_amax(qa, qb, mask)
+    D_plain = B.gemm(qa, qb, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    assert torch.equal(D.view(torch.int16), D_plain.view(torch.int16))
+    D_ref, norm = oracle.gemm_ref(*oracle.fprop_operands(X, W))
+    assert_gemm_close(D.float().cpu().numpy(), D_ref, norm, bf16=True, what="gemm_amax D")
+    qr, qc = B.quantize_row_rht(D, mask, 0)
+    got = amax.cpu().numpy().view(np.uint32)
+    want = np.array([qr.amax.item(), qc.amax.item()], dtype=np.float32).view(np.uint32)
+    assert np.array_equal(got, want), (got, want)
+
+
+@pytest.mark.parametrize("sr", [False, True])
+def test_quantizing_with_the_fused_maxima_changes_nothing(sr):
+    _, _, qa, qb = _operands(512, 1024, 768, seed=51)
+    mask = oracle.sign_mask_from_seed(51)
+    D, amax = B.gemm_amax(qa, qb, mask)
+    flags = B.SR if sr else 0
+    want_r, want_c = B.quantize_row_rht(D, mask, flags, seed=9, offset=4)
+    got_r, got_c = B.QuantizedTensor(*D.shape), B.QuantizedTensor(D.shape[1], D.shape[0])
+    got_r.amax.copy_(amax[0:1])
+    got_c.amax.copy_(amax[1:2])
+    B.quantize_row_rht(D, mask, flags | B.AMAX_GIVEN, seed=9, offset=4, out_row=got_r,
+                       out_col=got_c)
+    for got, want in ((got_r, want_r), (got_c, want_c)):
+        assert torch.equal(got.codes, want.codes)
+        assert torch.equal(got.scales, want.scales)
+        assert torch.equal(got.amax, want.amax)
+
+
+def test_gemm_amax_rejects_a_null_amax_buffer():
+    _, _, qa, qb = _operands(256, 256, 256, seed=52)
+    out = torch.empty((256, 256), dtype=torch.bfloat16, device="cuda")
+    oa, ob = qa.operand(), qb.operand()
+    st = B.lib().nvfp4_gemm_amax(ctypes.byref(oa), ctypes.byref(ob),
+                                 ctypes.c_void_p(out.data_ptr()), 256, 0, None, None, None)
+    assert st == B.ERR_NULL
