@@ -47,6 +47,9 @@ def lib():
                                    ctypes.c_int, ctypes.c_int, u64, u64, ctypes.c_int, fp,
                                    vp, vp, ctypes.POINTER(fp)]
         L.nvo_quantize.restype = ctypes.c_int
+        L.nvo_amax.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, u16,
+                               ctypes.POINTER(fp)]
+        L.nvo_amax.restype = ctypes.c_int
         L.nvo_dequantize.argtypes, L.nvo_dequantize.restype = [vp, vp, fp, i64, i64, vp], None
         L.nvo_gemm_ref.argtypes, L.nvo_gemm_ref.restype = [vp, vp, i64, i64, i64, vp], None
         L.nvo_row_norms.argtypes, L.nvo_row_norms.restype = [vp, i64, i64, vp], None
@@ -186,6 +189,19 @@ def quantize(x_bf16: np.ndarray, *, transpose=False, rht=False, sign_mask=0, blo
     if st not in (NVO_OK, NVO_ERR_NONFINITE):
         raise ValueError(f"oracle quantize rejected the arguments (status {st})")
     return Quantized(codes, scales, amax_out.value, st)
+
+
+def amax(x_bf16: np.ndarray, *, transpose=False, rht=False, sign_mask=0):
+    """The tensor amax ``quantize`` would compute for the same arguments (its first pass), on
+    its own and without materialising x^T: returns (amax, status)."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    out = ctypes.c_float(0.0)
+    st = lib().nvo_amax(_ptr(x), rows, cols, cols, int(transpose), int(rht), sign_mask,
+                        ctypes.byref(out))
+    if st not in (NVO_OK, NVO_ERR_NONFINITE):
+        raise ValueError(f"oracle amax rejected the arguments (status {st})")
+    return out.value, st
 
 
 # ---- MXFP4, the comparison format ------------------------------------------------------

@@ -282,6 +282,47 @@ static void build_rows(const uint16_t* x, int64_t ld, int transpose, int rht,
     }
 }
 
+/* The tensor amax alone: max |L| over the logical matrix L that nvo_quantize quantizes
+ * (x or its transpose; with `rht`, every 16-element block along L's rows replaced by its
+ * random Hadamard transform), i.e. the first pass of nvo_quantize [P1 Formato NVFP4: the
+ * tensor scale comes from the amax of the whole tensor].  x is walked in its own row order,
+ * 16 rows at a time when the blocks run down its columns, and x^T is never materialised, so
+ * the amax of a tensor too large to quantize on the CPU can still be had.  The value equals
+ * nvo_quantize's: the elements are the same, each transformed block is the same 16 values
+ * through nvo_rht16, and a maximum does not depend on the order it visits them.  Any NaN or
+ * Inf gives NVO_ERR_NONFINITE and amax +Inf, as in nvo_quantize. */
+int nvo_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int transpose, int rht,
+             uint16_t sign_mask, float* amax_out)
+{
+    if (rows <= 0 || cols <= 0) return NVO_ERR_ARG;
+    if (rht && (transpose ? rows : cols) % 16 != 0) return NVO_ERR_ARG;
+    float amax = 0.0f;
+    int nonfinite = 0;
+    float v[16], y[16];
+    /* one visit: a single element, or (rht) one block -- 16 values along x's row when L = x,
+     * down x's column when L = x^T */
+    for (int64_t r = 0; r < rows; r += (rht && transpose) ? 16 : 1) {
+        for (int64_t c = 0; c < cols; c += (rht && !transpose) ? 16 : 1) {
+            int m = 1;
+            if (!rht) {
+                y[0] = bf16_to_f32(x[r * ld + c]);
+            } else {
+                for (int i = 0; i < 16; ++i)
+                    v[i] = bf16_to_f32(transpose ? x[(r + i) * ld + c] : x[r * ld + c + i]);
+                nvo_rht16(v, sign_mask, y);
+                m = 16;
+            }
+            for (int i = 0; i < m; ++i) {
+                float a = fabsf(y[i]);
+                if (!isfinite(a)) nonfinite = 1;
+                else if (a > amax) amax = a;
+            }
+        }
+    }
+    *amax_out = nonfinite ? INFINITY : amax;
+    return nonfinite ? NVO_ERR_NONFINITE : NVO_OK;
+}
+
 /* Quantize a bf16 matrix x (rows x cols, row stride ld elements) to NVFP4 along the
  * logical rows of L (see build_rows).
  *

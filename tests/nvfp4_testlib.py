@@ -21,12 +21,13 @@ def to_device_bf16(bits: np.ndarray) -> torch.Tensor:
     return t.view(torch.bfloat16).cuda()
 
 
-def sf_offsets(rows: int, cols: int) -> np.ndarray:
+def sf_offsets(rows: int, cols: int, r=None, j=None) -> np.ndarray:
     """Byte offset of scale (r, j) in the MMA layout: 512-byte tiles of 128 rows x 4 blocks,
-    ordered (row tile, block group); inside a tile (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4."""
+    ordered (row tile, block group); inside a tile (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4.
+    All rows x all blocks, or the given row indices r x block indices j."""
     nb = cols // 16
-    r = np.arange(rows, dtype=np.int64)[:, None]
-    j = np.arange(nb, dtype=np.int64)[None, :]
+    r = np.arange(rows, dtype=np.int64)[:, None] if r is None else np.asarray(r, np.int64)[:, None]
+    j = np.arange(nb, dtype=np.int64)[None, :] if j is None else np.asarray(j, np.int64)[None, :]
     return ((r // 128) * (nb // 4) + j // 4) * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + j % 4
 
 
