@@ -482,11 +482,12 @@ def run_kernel_case(args):
     T, D, F = 8192, 5120, 20480
     dev = torch.device("cuda", torch.cuda.current_device())
     ws = torch.empty((B.workspace_bytes(1 << 14, 1 << 14),), dtype=torch.uint8, device=dev)
-    if args.kernel in ("gemm", "gemm_amax", "chain", "chain_amax"):
+    if args.kernel in ("gemm", "gemm_amax", "chain", "chain_amax", "gemm_mx"):
         X = torch.from_numpy(synth.activations((T, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
         W = torch.from_numpy(synth.weights((F, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
-        qa, _ = B.quantize(X, B.ROWWISE, workspace=ws)
-        qb, _ = B.quantize(W, B.ROWWISE | B.BLOCK2D, workspace=ws)
+        mx = B.MX if args.kernel == "gemm_mx" else 0
+        qa, _ = B.quantize(X, B.ROWWISE | mx, workspace=ws)
+        qb, _ = B.quantize(W, B.ROWWISE | (mx or B.BLOCK2D), workspace=ws)
         out = torch.empty((T, F), dtype=torch.bfloat16, device=dev)
         amax = torch.empty(2, dtype=torch.float32, device=dev)
         qr, qc = B.QuantizedTensor(T, F, dev), B.QuantizedTensor(F, T, dev)
@@ -506,10 +507,12 @@ def run_kernel_case(args):
 
         fn = {"gemm": lambda: B.gemm(qa, qb, out=out),
               "gemm_amax": lambda: B.gemm_amax(qa, qb, 0x5A3C, out=out, amax_out=amax),
-              "chain": chain, "chain_amax": chain_amax}[args.kernel]
+              "chain": chain, "chain_amax": chain_amax,
+              "gemm_mx": lambda: B.gemm(qa, qb, out=out, mx=True)}[args.kernel]
         work, unit, peak = 2 * T * D * F / 1e12, "TFLOP/s", peaks["bf16_tflops"] * FP4_OVER_BF16
         shape = f"M={T} N={F} K={D}, bf16 out" + (
-            ", then SR dual quantization of D" if args.kernel.startswith("chain") else "")
+            ", then SR dual quantization of D" if args.kernel.startswith("chain") else "") + (
+            ", MXFP4 operands" if mx else "")
     else:
         x = torch.from_numpy(synth.gradients((T, F), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
         n = T * F
@@ -522,6 +525,13 @@ def run_kernel_case(args):
         elif args.kernel == "rht":
             q = B.QuantizedTensor(F, T, dev)
             fn = lambda: B.rht_quantize(x, 0x5A3C, B.SR, seed=1, out_col=q, workspace=ws)  # noqa: E731
+        elif args.kernel == "rowwise_mx":
+            q = B.QuantizedTensor(T, F, dev)
+            fn = lambda: B.quantize(x, B.ROWWISE | B.MX, out_row=q, workspace=ws)  # noqa: E731
+        elif args.kernel == "rht_mx":
+            q = B.QuantizedTensor(F, T, dev)
+            fn = lambda: B.rht_quantize(x, 0x5A3C, B.SR | B.MX, seed=1, out_col=q,  # noqa: E731
+                                        workspace=ws)
         else:
             q = B.QuantizedTensor(T, F, dev)
             q2 = B.QuantizedTensor(F, T, dev)
@@ -700,8 +710,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["gemm", "gemm_amax", "chain", "chain_amax", "rowwise",
-                                         "tile2d", "rht", "dual"], default=None,
+    ap.add_argument("--kernel", choices=["gemm", "gemm_amax", "chain", "chain_amax", "gemm_mx",
+                                         "rowwise", "tile2d", "rht", "dual", "rowwise_mx",
+                                         "rht_mx"], default=None,
                     help="time one kernel family alone at the workload's shapes (profiling)")
     ap.add_argument("--sweep", action="store_true",
                     help="quantizer bandwidth sweep over 2^n-element tensors (one line per point)")
