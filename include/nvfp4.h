@@ -220,8 +220,10 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
  *   amax_out : device, 2 FP32 (4-byte aligned), overwritten: amax_out[0] = max |D| and
  *              amax_out[1] = max |RHT(D)| (16x16 transform of every 16 consecutive rows of each
  *              column with sign_mask), both over D as stored in bf16 -- exactly the amax values
- *              nvfp4_quantize_row_rht(D, sign_mask) computes.  NaN or Inf in D gives a value
- *              at or above +Inf.
+ *              nvfp4_quantize_row_rht(D, sign_mask) computes.  NaN or Inf in D makes the
+ *              maximum +Inf or a NaN (the maxima are taken on the magnitude bit patterns), which
+ *              the quantizer then treats as non-finite data: zero outputs and
+ *              NVFP4_DEVSTAT_NONFINITE, as without the fused maxima.
  * Pass them to nvfp4_quantize_row_rht with NVFP4_AMAX_GIVEN (out_row->amax = &amax_out[0],
  * out_col->amax = &amax_out[1]) to skip its amax pass.  Other arguments as nvfp4_gemm.
  */
