@@ -7,23 +7,25 @@
 // Design (one CTA per SM, persistent over 128 x 256 output tiles, 22 warps):
 //   warp 0      TMA producer: per 256-wide K block, the A (128 x 128 B) and B (256 x 128 B)
 //               code tiles with 128-byte swizzle, plus the block scales (contiguous 512-byte
-//               tiles of the MMA scale layout) by bulk copies; a shared-memory ring of 4
-//               stages (bf16 output) or 3 (FP32 output) guarded by mbarriers.  One stage's
-//               round trip (TMA ~1.7 k cycles, scale staging ~0.55 k, issue ~0.5 k, MMAs +
-//               release ~1.1 k) is about four stages of MMA work, so with three stages the
-//               tensor pipe idles about a third of the time.
+//               tiles of the MMA scale layout) by bulk copies, into a shared-memory ring of 4
+//               stages guarded by mbarriers.  The four MMAs of a stage take ~0.54 k cycles on
+//               the tensor pipe, while a stage's round trip (TMA ~1.7 k, scale staging
+//               ~0.55 k, issue ~0.5 k, MMAs + release ~1.1 k, more under load) spans several
+//               stages' MMA work: the kernel is bound by this operand feed, not by the MMAs.
 //   warps 2-5   scale stagers, one per 32-lane quarter of tensor memory: move each stage's
 //               scales shared -> registers -> tensor memory (ld.shared + tcgen05.st, into a
 //               per-stage column range), so the tensor pipe never spends time on scale copies.
 //   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::mxf4nvf4 (M 128,
-//               N 256, K 64, FP32 accumulation in TMEM), then commits the stage back to the
-//               producer.
+//               N 256, K 64, FP32 accumulation in TMEM; E4M3 scales, or UE8M0 for MXFP4
+//               operands), then commits the stage back to the producer.
 //   warps 6-21  epilogue: each warp drains one 32-lane quarter x 64 columns of the
 //               accumulator into registers (tcgen05.ld), releases the accumulator so the
 //               next tile's MMAs start at once, then scales by 1 / (S_enc,A S_enc,B) and
-//               writes FP32 or bf16 rows through a per-warp shared-memory staging buffer
-//               with paced TMA bulk tensor stores (clipped at the matrix edge) while the next
-//               tile computes.
+//               writes the tile while the next one computes: bf16 rows through a 512-byte
+//               per-warp staging buffer with paced TMA bulk tensor stores (clipped at the
+//               matrix edge), FP32 pairs straight from registers with 8-byte stores.  With
+//               the fused amax, the bf16 epilogue also reduces max |D| and, by 16-lane
+//               shuffles across rows, max |RHT(D)| for the next quantization of D.
 // Every wait on an mbarrier is bounded in time; on expiry the kernel records
 // NVFP4_DEVSTAT_TIMEOUT, drains its in-flight copies and MMAs (again with a limit), frees
 // its tensor memory and returns.
