@@ -6,15 +6,19 @@
 // fixed random sign vector on the weight-gradient inputs) and "Escalado Bidimensional (2D)
 // y Redondeo Estocastico" (16x16 weight blocks; stochastic rounding of gradients).
 //
-// Two passes over the bf16 input, both HBM-bound streams:
-//   1. amax_kernel / amax_rht_kernel: per-CTA partial maxima of |x| (or |RHT(x)|) into the
-//      workspace.  The plain pass compares bf16 magnitude bit patterns (exact).
+// Two passes over the bf16 input (streams bound by HBM when rounding to nearest, by
+// instruction issue with stochastic rounding):
+//   1. amax_kernel / amax_rht_kernel: per-CTA partial maxima of |x| (or |RHT(x)|, or both
+//      for the one-pass pair) into the workspace.  The plain pass compares bf16 magnitude
+//      bit patterns (exact).
 //   2. quant_rowwise_kernel (1x16 blocks along the row, coalesced 16-byte loads, block max
 //      by one warp shuffle, one Philox call per 8 elements for SR) or quant_tile_kernel
 //      (64 x 128 tiles staged in shared memory for the column-wise / transposed outputs,
-//      16x16 weight tiles and the fused RHT).  Each CTA first folds the partial maxima into
-//      the tensor amax.  The second pass walks the tensor in the reverse order of the
-//      first, so the tail the first pass left in L2 is re-read from L2.
+//      16x16 weight tiles, the fused RHT, the one-pass pair of a tensor's row-wise and RHT'd
+//      column-wise outputs, and the MXFP4 variant's 32-element blocks).  Each CTA first
+//      folds the partial maxima into the tensor amax.  The second pass walks the tensor in
+//      the reverse order of the first, so the tail the first pass left in L2 is re-read
+//      from L2.
 #include <cuda_runtime.h>
 
 #include <cstdint>
