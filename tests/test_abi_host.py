@@ -160,6 +160,37 @@ def test_gemm_argument_validation(case, expected):
     assert L.nvfp4_gemm(ctypes.byref(A), ctypes.byref(Bo), D, dt, ldd, None, None) == expected
 
 
+def test_gemm_amax_argument_validation():
+    """nvfp4_gemm_amax: bf16 output only, a 4-byte-aligned amax_out pair, the GEMM's shape
+    rules; a valid call without a GPU fails with a CUDA/device status, never a crash."""
+    L = B.lib()
+    A, Bo = _op(256, 512), _op(384, 512, base=0x400000)
+    D, amax = ctypes.c_void_p(0x9000), ctypes.c_void_p(0xA000)
+    assert L.nvfp4_gemm_amax(ctypes.byref(A), ctypes.byref(Bo), D, 384, 0, None, None,
+                             None) == B.ERR_NULL
+    assert L.nvfp4_gemm_amax(ctypes.byref(A), ctypes.byref(Bo), D, 384, 0,
+                             ctypes.c_void_p(0xA002), None, None) == B.ERR_ALIGN
+    # bf16 rows: ldd * 2 bytes must be a multiple of 16
+    assert L.nvfp4_gemm_amax(ctypes.byref(A), ctypes.byref(Bo), D, 388, 0, amax, None,
+                             None) == B.ERR_ALIGN
+    assert L.nvfp4_gemm_amax(ctypes.byref(A), ctypes.byref(_op(384, 448, base=0x400000)), D,
+                             384, 0, amax, None, None) == B.ERR_SHAPE
+    assert L.nvfp4_gemm_amax(ctypes.byref(A), ctypes.byref(Bo), D, 384, 0x1234, amax, None,
+                             None) in (B.ERR_CUDA, B.ERR_DEVICE)
+
+
+def test_gemm_mx_argument_validation():
+    L = B.lib()
+    A, Bo = _op(256, 512), _op(384, 512, base=0x400000)
+    D = ctypes.c_void_p(0x9000)
+    assert L.nvfp4_gemm_mx(ctypes.byref(A), ctypes.byref(_op(384, 96, base=0x400000)), D,
+                           B.OUT_F32, 384, None, None) == B.ERR_SHAPE
+    assert L.nvfp4_gemm_mx(ctypes.byref(A), ctypes.byref(Bo), None, B.OUT_F32, 384, None,
+                           None) == B.ERR_NULL
+    assert L.nvfp4_gemm_mx(ctypes.byref(A), ctypes.byref(Bo), D, 5, 384, None,
+                           None) == B.ERR_ARG
+
+
 def test_linear_argument_validation():
     L = B.lib()
     p = ctypes.c_void_p(0x1000)
