@@ -285,6 +285,29 @@ nvfp4_status nvfp4_linear_wgrad(const void* dY, const void* X, int64_t T, int64_
                                 int dw_dtype, void* workspace, int* dev_status, void* stream);
 
 /*
+ * nvfp4_linear_dgrad with bf16 output, also quantized for the previous layer's backward pass:
+ * dX = dY . W and dX's two NVFP4 operands, the ones the previous layer's dgrad and wgrad read
+ * (dX is that layer's output gradient) [P1 Escalado 2D y Redondeo Estocastico; P1 RHT]:
+ *   dX_row : T x I along I, 1x16 SR on stream next_offset;
+ *   dX_col : I x T along T, RHT + 1x16 SR on stream next_offset + 1;
+ * bit for bit what nvfp4_linear_dgrad(..., NVFP4_OUT_BF16) followed by
+ * nvfp4_quantize_row_rht(dX, sign_mask, NVFP4_SR, next_seed, next_offset) writes, including
+ * each operand's amax.  The GEMM epilogue emits dX's two maxima (nvfp4_gemm_amax), so dX is
+ * quantized without an amax pass.
+ *   dX_bf16   : device, T x I bf16, row stride I.
+ *   dX_row, dX_col : the caller's operands (shapes as above); checked before any work is
+ *               queued, like every other argument.
+ *   workspace : nvfp4_linear_workspace_bytes(T, I, O) device bytes.
+ * Shape rules: T, I, O multiples of 64.
+ */
+nvfp4_status nvfp4_linear_dgrad_quantized(const void* dY, const void* W, int64_t T, int64_t I,
+                                          int64_t O, uint64_t seed, uint64_t offset,
+                                          void* dX_bf16, uint16_t sign_mask, uint64_t next_seed,
+                                          uint64_t next_offset, const nvfp4_operand* dX_row,
+                                          const nvfp4_operand* dX_col, void* workspace,
+                                          int* dev_status, void* stream);
+
+/*
  * nvfp4_quantize without a caller workspace, for callers that cannot allocate device memory
  * where they quantize (a host framework that owns all device memory through its own
  * fixed arena, or a latency-critical loop that must not enter cudaMalloc / cudaFree, which may

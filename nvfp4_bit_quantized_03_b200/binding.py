@@ -80,6 +80,9 @@ def lib():
         L.nvfp4_linear_dgrad.restype = i32
         L.nvfp4_linear_wgrad.argtypes = [vp, vp, i64, i64, i64, u16, u64, u64, vp, i32, vp, vp, vp]
         L.nvfp4_linear_wgrad.restype = i32
+        L.nvfp4_linear_dgrad_quantized.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, u16, u64,
+                                                   u64, op, op, vp, vp, vp]
+        L.nvfp4_linear_dgrad_quantized.restype = i32
         _lib = L
     return _lib
 
@@ -301,6 +304,33 @@ def linear_dgrad(dY, W, seed, offset, out=None, out_dtype=torch.float32, workspa
                                   _stream(stream))
     _check(st, "nvfp4_linear_dgrad")
     return out
+
+
+def linear_dgrad_quantized(dY, W, seed, offset, sign_mask, next_seed, next_offset, out=None,
+                           out_row=None, out_col=None, workspace=None, dev_status=None,
+                           stream=None):
+    """nvfp4_linear_dgrad_quantized: bf16 dX = dY . W plus dX's row-wise SR and RHT'd
+    column-wise SR operands for the previous layer (returns dX, dX_row, dX_col)."""
+    T, O = dY.shape
+    I = W.shape[1]
+    if out is None:
+        out = torch.empty((T, I), dtype=torch.bfloat16, device=dY.device)
+    _check_out(out, T, I, "nvfp4_linear_dgrad_quantized")
+    if out.dtype != torch.bfloat16:
+        raise TypeError("nvfp4_linear_dgrad_quantized: dX must be bfloat16")
+    if out_row is None:
+        out_row = QuantizedTensor(T, I, dY.device)
+    if out_col is None:
+        out_col = QuantizedTensor(I, T, dY.device)
+    if workspace is None:
+        workspace = _workspace(linear_workspace_bytes(T, I, O), dY.device)
+    op_r, op_c = out_row.operand(), out_col.operand()
+    st = lib().nvfp4_linear_dgrad_quantized(_ptr(dY), _ptr(W), T, I, O, seed, offset, _ptr(out),
+                                            sign_mask, next_seed, next_offset,
+                                            ctypes.byref(op_r), ctypes.byref(op_c),
+                                            _ptr(workspace), _ptr(dev_status), _stream(stream))
+    _check(st, "nvfp4_linear_dgrad_quantized")
+    return out, out_row, out_col
 
 
 def linear_wgrad(dY, X, sign_mask, seed, offset, out=None, out_dtype=torch.float32,

@@ -469,6 +469,46 @@ nvfp4_status nvfp4_linear_dgrad(const void* dY, const void* W, int64_t T, int64_
     return nvfp4_gemm(&w.a, &w.b, dX, dx_dtype, I, dev_status, stream);
 }
 
+nvfp4_status nvfp4_linear_dgrad_quantized(const void* dY, const void* W, int64_t T, int64_t I,
+                                          int64_t O, uint64_t seed, uint64_t offset,
+                                          void* dX_bf16, uint16_t sign_mask, uint64_t next_seed,
+                                          uint64_t next_offset, const nvfp4_operand* dX_row,
+                                          const nvfp4_operand* dX_col, void* workspace,
+                                          int* dev_status, void* stream)
+{
+    // every argument is checked before the first kernel is queued
+    nvfp4_status st = check_linear(dY, W, dX_bf16, workspace, T, I, O, NVFP4_OUT_BF16);
+    if (st != NVFP4_OK) return st;
+    if ((st = check_operand(dX_row, T, I)) != NVFP4_OK) return st;
+    if ((st = check_operand(dX_col, I, T)) != NVFP4_OK) return st;
+    LinearWorkspace w = carve(workspace, T, O, I, O);
+    if ((st = nvfp4_quantize(W, O, I, I, NVFP4_COLWISE | NVFP4_BLOCK2D, 0, 0, nullptr, &w.b,
+                             w.partials, dev_status, stream)) != NVFP4_OK)
+        return st;
+    if ((st = nvfp4_quantize(dY, T, O, O, NVFP4_ROWWISE | NVFP4_SR, seed, offset, &w.a, nullptr,
+                             w.partials, dev_status, stream)) != NVFP4_OK)
+        return st;
+    // dX and its two maxima from the epilogue, into the partials area (the quantize kernels
+    // that used it are ahead on the stream)
+    float* maxima = static_cast<float*>(w.partials);
+    if ((st = nvfp4_gemm_amax(&w.a, &w.b, dX_bf16, I, sign_mask, maxima, dev_status, stream)) !=
+        NVFP4_OK)
+        return st;
+    nvfp4_operand r = *dX_row, c = *dX_col;
+    r.amax = maxima;
+    c.amax = maxima + 1;
+    if ((st = nvfp4_quantize_row_rht(dX_bf16, T, I, I, sign_mask,
+                                     NVFP4_SR | NVFP4_AMAX_GIVEN, next_seed, next_offset, &r, &c,
+                                     nullptr, dev_status, stream)) != NVFP4_OK)
+        return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if ((st = from_cuda(cudaMemcpyAsync(dX_row->amax, maxima, sizeof(float),
+                                        cudaMemcpyDeviceToDevice, s))) != NVFP4_OK)
+        return st;
+    return from_cuda(cudaMemcpyAsync(dX_col->amax, maxima + 1, sizeof(float),
+                                     cudaMemcpyDeviceToDevice, s));
+}
+
 nvfp4_status nvfp4_linear_wgrad(const void* dY, const void* X, int64_t T, int64_t I, int64_t O,
                                 uint16_t sign_mask, uint64_t seed, uint64_t offset, void* dW,
                                 int dw_dtype, void* workspace, int* dev_status, void* stream)

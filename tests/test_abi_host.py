@@ -179,6 +179,15 @@ def test_gemm_amax_argument_validation():
                              None) in (B.ERR_CUDA, B.ERR_DEVICE)
 
 
+def test_dgrad_quantized_argument_validation():
+    L = B.lib()
+    p = ctypes.c_void_p(0x1000)
+    assert L.nvfp4_linear_dgrad_quantized(p, p, 256, 512, 384, 0, 0, p, 0, 0, 0, None, None,
+                                          None, None, None) == B.ERR_NULL
+    assert L.nvfp4_linear_dgrad_quantized(p, p, 100, 512, 384, 0, 0, p, 0, 0, 0, None, None,
+                                          p, None, None) == B.ERR_SHAPE
+
+
 def test_gemm_mx_argument_validation():
     L = B.lib()
     A, Bo = _op(256, 512), _op(384, 512, base=0x400000)

@@ -78,3 +78,41 @@ def test_gemm_amax_rejects_a_null_amax_buffer():
     st = B.lib().nvfp4_gemm_amax(ctypes.byref(oa), ctypes.byref(ob),
                                  ctypes.c_void_p(out.data_ptr()), 256, 0, None, None, None)
     assert st == B.ERR_NULL
+
+
+@pytest.mark.parametrize("T,I,O", [(256, 512, 384), (1024, 2048, 1536)])
+def test_dgrad_quantized_equals_the_unfused_sequence(T, I, O):
+    """nvfp4_linear_dgrad_quantized = nvfp4_linear_dgrad (bf16) then nvfp4_quantize_row_rht
+    (SR) of its dX, bit for bit: dX, both operands' codes and scales, and their amax."""
+    dY = synth.gradients((T, O), seed=53)
+    W = synth.weights((O, I), seed=53)
+    dYd, Wd = to_device_bf16(dY), to_device_bf16(W)
+    mask = oracle.sign_mask_from_seed(53)
+    dX_ref = B.linear_dgrad(dYd, Wd, 3, 1, out_dtype=torch.bfloat16)
+    qr_ref, qc_ref = B.quantize_row_rht(dX_ref, mask, B.SR, seed=11, offset=5)
+    dX, qr, qc = B.linear_dgrad_quantized(dYd, Wd, 3, 1, mask, 11, 5)
+    torch.cuda.synchronize()
+    assert torch.equal(dX.view(torch.int16), dX_ref.view(torch.int16))
+    for got, want in ((qr, qr_ref), (qc, qc_ref)):
+        assert torch.equal(got.codes, want.codes)
+        assert torch.equal(got.scales, want.scales)
+        assert torch.equal(got.amax, want.amax)
+    D_ref, norm = oracle.gemm_ref(*oracle.dgrad_operands(dY, W, 3, 1))
+    assert_gemm_close(dX.float().cpu().numpy(), D_ref, norm, bf16=True, what="dgrad_quantized dX")
+
+
+def test_dgrad_quantized_rejects_bad_operands():
+    T, I, O = 256, 512, 384
+    dYd = to_device_bf16(synth.gradients((T, O), seed=54))
+    Wd = to_device_bf16(synth.weights((O, I), seed=54))
+    with pytest.raises(B.NVFP4Error) as e:
+        B.linear_dgrad_quantized(dYd, Wd, 0, 0, 0, 0, 0, out_col=B.QuantizedTensor(T, I))
+    assert e.value.status == B.ERR_SHAPE
+    dX = torch.empty((T, I), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty((B.linear_workspace_bytes(T, I, O),), dtype=torch.uint8, device="cuda")
+    oc = B.QuantizedTensor(I, T).operand()
+    st = B.lib().nvfp4_linear_dgrad_quantized(
+        ctypes.c_void_p(dYd.data_ptr()), ctypes.c_void_p(Wd.data_ptr()), T, I, O, 0, 0,
+        ctypes.c_void_p(dX.data_ptr()), 0, 0, 0, None, ctypes.byref(oc),
+        ctypes.c_void_p(ws.data_ptr()), None, None)
+    assert st == B.ERR_NULL
