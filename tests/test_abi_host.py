@@ -86,6 +86,9 @@ def _op(rows, cols, base=0x10000):
     ("out_shape", B.ERR_SHAPE),
     ("out_null_codes", B.ERR_NULL),
     ("no_workspace", B.ERR_NULL),
+    ("empty", B.ERR_SHAPE),
+    ("negative_cols", B.ERR_SHAPE),
+    ("too_large", B.ERR_SHAPE),
 ])
 def test_quantize_argument_validation(case, expected):
     L = B.lib()
@@ -120,6 +123,12 @@ def test_quantize_argument_validation(case, expected):
         out_row = B.Operand(0, 0x2000, 0x3000, 256, 512)
     elif case == "no_workspace":
         ws = None
+    elif case == "empty":
+        rows, out_row = 0, _op(0, 512)
+    elif case == "negative_cols":
+        cols, out_row = -512, _op(256, -512)
+    elif case == "too_large":
+        rows, out_row = 1 << 31, _op(1 << 31, 512)
     out_col = _op(cols, rows) if flags & B.COLWISE else None
     st = L.nvfp4_quantize(x, rows, cols, ld, flags, 0, 0,
                           ctypes.byref(out_row) if flags & B.ROWWISE else None,
@@ -138,7 +147,7 @@ def test_rht_quantize_rejects_rowwise_flags():
 @pytest.mark.parametrize("case,expected", [
     ("k_mismatch", B.ERR_SHAPE), ("k_not_64", B.ERR_SHAPE), ("m_not_16", B.ERR_SHAPE),
     ("ldd_small", B.ERR_SHAPE), ("ldd_unaligned", B.ERR_ALIGN), ("dtype", B.ERR_ARG),
-    ("null_d", B.ERR_NULL)])
+    ("null_d", B.ERR_NULL), ("m_zero", B.ERR_SHAPE), ("k_too_large", B.ERR_SHAPE)])
 def test_gemm_argument_validation(case, expected):
     L = B.lib()
     A, Bo = _op(256, 512), _op(384, 512, base=0x400000)
@@ -157,6 +166,10 @@ def test_gemm_argument_validation(case, expected):
         dt = 7
     elif case == "null_d":
         D = None
+    elif case == "m_zero":
+        A = _op(0, 512)
+    elif case == "k_too_large":
+        A, Bo = _op(256, 1 << 31), _op(384, 1 << 31, base=0x400000)
     assert L.nvfp4_gemm(ctypes.byref(A), ctypes.byref(Bo), D, dt, ldd, None, None) == expected
 
 
