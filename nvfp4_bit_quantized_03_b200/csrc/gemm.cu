@@ -303,12 +303,56 @@ __device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t* v)
 }
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Tensor encode scale of an operand, as the quantizer computed it; see alpha below.
+// Tensor encode scale of an operand, as the quantizer computed it; see Alpha below.
 __device__ __forceinline__ float operand_scale(float amax)
 {
     if (amax == 0.0f) return 1.0f;
     const float s = __fdiv_rn(2688.0f, amax);
     return s > FLT_MAX ? FLT_MAX : s;
+}
+
+// The epilogue's decode factor 1 / (S_enc,A S_enc,B), applied as two FP32 multiplies
+// D = (acc * a1) * a2.  The product of two FP32 encode scales spans 2^-256 .. 2^256, beyond
+// FP32, so it is formed in FP64 (the 24 x 24-bit product is exact, the reciprocal rounded
+// once) and split into a1 = m 2^e1 (m in [1, 2), e1 = e clamped to [-100, 70]) and the power
+// of two a2 = 2^(e - e1).  A non-zero accumulator lies in [2^-20, 2^54] (products of E2M1
+// values, at least 1/2, and E4M3 scales, at least 2^-9; K < 2^31 terms of at most 6^2 448^2),
+// so acc * a1 is always a normal FP32 value and the only rounding that matters is the last
+// one.  When e - e1 falls outside [-149, 127] it is clamped: then every non-zero |acc| / (S_A
+// S_B) is below 2^-194 or above 2^177, and the clamped product rounds to the same 0 or Inf.
+// Non-finite operands (amax = Inf) give 0; MXFP4 operands carry no tensor scale (a1 = a2 = 1).
+struct Alpha {
+    float a1, a2;
+};
+
+__device__ __forceinline__ float pow2f(int e)  // 2^e for e in [-149, 127], exact
+{
+    return e >= -126 ? __uint_as_float(static_cast<uint32_t>(e + 127) << 23)
+                     : __uint_as_float(1u << (e + 149));
+}
+
+template <bool MX>
+__device__ __forceinline__ Alpha epilogue_alpha(float amax_a, float amax_b)
+{
+    const bool finite = (amax_a < INFINITY) && (amax_b < INFINITY) && amax_a >= 0.0f &&
+                        amax_b >= 0.0f;
+    if (!finite) return Alpha{0.0f, 1.0f};
+    if (MX) return Alpha{1.0f, 1.0f};
+    const double alpha = 1.0 / (static_cast<double>(operand_scale(amax_a)) *
+                                static_cast<double>(operand_scale(amax_b)));
+    const int e = static_cast<int>((__double_as_longlong(alpha) >> 52) & 0x7FF) - 1023;
+    const int e1 = e < -100 ? -100 : (e > 70 ? 70 : e);
+    int e2 = e - e1;
+    e2 = e2 < -149 ? -149 : (e2 > 127 ? 127 : e2);
+    // alpha * 2^-(e - e1) by exponent arithmetic on the FP64 pattern (exact), then to FP32
+    const double scaled = __longlong_as_double(__double_as_longlong(alpha) -
+                                               (static_cast<long long>(e - e1) << 52));
+    return Alpha{__double2float_rn(scaled), pow2f(e2)};
+}
+
+__device__ __forceinline__ float apply_alpha(uint32_t acc_bits, const Alpha& al)
+{
+    return __fmul_rn(__fmul_rn(__uint_as_float(acc_bits), al.a1), al.a2);
 }
 
 // Output tile order: groups of 16 row tiles, column tiles inner, so that the CTAs working
@@ -342,7 +386,7 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 // lane keeping a + b and the upper a - b -- the same FP32 operations, in the same order, as the
 // quantizer's transform of the bf16 values.
 template <bool BF16, bool AMAX = false>
-__device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint32_t stage_buf,
+__device__ __forceinline__ void store_slice(const uint32_t* v, const Alpha& alpha, uint32_t stage_buf,
                                             int lane, const CUtensorMap* tmap_d, int n0, int y,
                                             int M, int N, uint32_t* m_plain = nullptr,
                                             uint32_t* m_rht = nullptr, uint32_t flip = 0)
@@ -366,8 +410,7 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint
                 for (int h = 0; h < 4; ++h) {
                     const int j = r * 8 + 2 * h;
                     const __nv_bfloat162 b2 =
-                        __floats2bfloat162_rn(__fmul_rn(__uint_as_float(v[j]), alpha),
-                                              __fmul_rn(__uint_as_float(v[j + 1]), alpha));
+                        __floats2bfloat162_rn(apply_alpha(v[j], alpha), apply_alpha(v[j + 1], alpha));
                     o[h] = *reinterpret_cast<const uint32_t*>(&b2);
                 }
                 if (AMAX) {
@@ -394,7 +437,7 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint
             } else {
 #pragma unroll
                 for (int h = 0; h < 4; ++h)
-                    o[h] = __float_as_uint(__fmul_rn(__uint_as_float(v[r * 16 + c * 4 + h]), alpha));
+                    o[h] = __float_as_uint(apply_alpha(v[r * 16 + c * 4 + h], alpha));
             }
             asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_base + 16 * (c ^ swz)),
                          "r"(o[0]), "r"(o[1]), "r"(o[2]), "r"(o[3])
@@ -411,7 +454,7 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, float alpha, uint
 // tmem_ld_16x256b_x8 for the two 16-row halves): scaled by alpha, each instruction writes 8 B
 // per thread, i.e. 8 rows x 32 contiguous bytes (whole sectors) per warp; no staging, so the
 // FP32 kernel keeps the shared memory for operand stages like the bf16 one.
-__device__ __forceinline__ void store_f32_direct(const uint32_t* v, float alpha, float* D,
+__device__ __forceinline__ void store_f32_direct(const uint32_t* v, const Alpha& alpha, float* D,
                                                  int64_t ldd, int lane, int n0, int y, int M,
                                                  int N)
 {
@@ -425,8 +468,8 @@ __device__ __forceinline__ void store_f32_direct(const uint32_t* v, float alpha,
             for (int k = 0; k < 2; ++k) {
                 const int row = y + 16 * h + (lane >> 2) + 8 * k;
                 if (row < M && col < N) {
-                    const float2 val = make_float2(__fmul_rn(__uint_as_float(r[2 * k]), alpha),
-                                                   __fmul_rn(__uint_as_float(r[2 * k + 1]), alpha));
+                    const float2 val =
+                        make_float2(apply_alpha(r[2 * k], alpha), apply_alpha(r[2 * k + 1], alpha));
                     *reinterpret_cast<float2*>(D + static_cast<int64_t>(row) * ldd + col) = val;
                 }
             }
@@ -638,12 +681,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int q = warp & 3;                         // TMEM lane quarter this warp may access
         const int chunk = (warp - FIRST_EPI_WARP) >> 2; // accumulator columns [64 chunk, +64)
         const uint32_t stage_buf = smem_u32(staging + (warp - FIRST_EPI_WARP) * STAGING_BYTES);
-        const float aa = *p.amax_a, ab = *p.amax_b;
-        const bool finite = (aa < INFINITY) && (ab < INFINITY) && aa >= 0.0f && ab >= 0.0f;
         // NVFP4: undo both tensor scales; MXFP4 has none (its amax only flags bad data)
-        const float alpha =
-            !finite ? 0.0f
-                    : (MX ? 1.0f : __fdiv_rn(1.0f, __fmul_rn(operand_scale(aa), operand_scale(ab))));
+        const Alpha alpha = epilogue_alpha<MX>(*p.amax_a, *p.amax_b);
         int it = 0;
         uint32_t m_plain = 0, m_rht = 0;  // fused maxima (AMAX)
         const uint32_t flip = ((p.sign_mask >> (lane & 15)) & 1u) ? 0x80000000u : 0u;

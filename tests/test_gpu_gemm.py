@@ -8,7 +8,8 @@ import torch
 
 import oracle
 import synth
-from nvfp4_testlib import assert_gemm_close, need_gpu, upload_quantized
+from nvfp4_testlib import (assert_gemm_close, assert_quantized_equal, need_gpu,
+                           to_device_bf16, upload_quantized)
 
 nv = pytest.importorskip("nvfp4_bit_quantized_03_b200")
 B = nv.binding
@@ -89,3 +90,58 @@ def test_gemm_is_deterministic():
     d1 = B.gemm(A, Bq)
     d2 = B.gemm(A, Bq)
     assert torch.equal(d1, d2)
+
+
+def _scaled(bits, k):
+    """bf16 values times 2^k, exactly (every value stays a normal number or zero)."""
+    return synth.f32_to_bf16_bits(synth.bf16_bits_to_f32(bits) * np.float32(2.0 ** k))
+
+
+@pytest.mark.parametrize("ka,kb", [(-60, -60), (-70, -45), (-95, -25)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_gemm_extreme_amax(ka, kb, dtype):
+    """Operands whose tensor scales multiply beyond FP32 (S_A * S_B > FLT_MAX): inputs scaled
+    by tiny powers of two, quantized by the GPU (bit-exact with the oracle) and multiplied.
+    The decode factor 1 / (S_A S_B) must not collapse to 0: D is compared entry by entry with
+    the oracle's FP64 products of the dequantized operands."""
+    M, N, K = 256, 512, 512
+    X = _scaled(synth.activations((M, K), seed=70), ka)
+    W = _scaled(synth.weights((N, K), seed=70), kb)
+    qa_ref, qb_ref = oracle.quantize(X), oracle.quantize(W, block2d=True)
+    # the extreme case: the product of the two FP32 encode scales exceeds FLT_MAX
+    assert oracle.tensor_scale(qa_ref.amax) * oracle.tensor_scale(qb_ref.amax) > 3.4028235e38
+    qa, _ = B.quantize(to_device_bf16(X), B.ROWWISE)
+    qb, _ = B.quantize(to_device_bf16(W), B.ROWWISE | B.BLOCK2D)
+    assert_quantized_equal(qa, qa_ref, "A")
+    assert_quantized_equal(qb, qb_ref, "B")
+    D = B.gemm(qa, qb, out_dtype=dtype)
+    D_ref, norm = oracle.gemm_ref(qa_ref, qb_ref)
+    assert np.abs(D_ref).max() > 0
+    assert_gemm_close(D.float().cpu().numpy(), D_ref, norm, bf16=(dtype == torch.bfloat16),
+                      what=f"2^{ka} x 2^{kb}")
+
+
+@pytest.mark.parametrize("amax_a,amax_b,sf_hi", [
+    (2.0 ** 75.5, 2.0 ** 75.5, 4),      # S_A * S_B below FP32's normal range: 1/x overflows
+    (2.0 ** -60, 2.0 ** -60, 0x7E),     # S_A * S_B above FLT_MAX
+    (2.0 ** -126, 3.0e38, 0x7E),        # far apart, product ordinary
+    (1.0e-40, 1.0e-40, 0x7E),           # subnormal amax: both scales clamp to FLT_MAX
+])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_gemm_decode_factor_over_the_whole_amax_range(amax_a, amax_b, sf_hi, dtype):
+    """The GEMM's contract for arbitrary operands: D = sum_k deq(A) deq(B) with deq = e2m1 x
+    sf / S_enc(amax).  Random codes, random scale bytes in [1, sf_hi] and a chosen amax per
+    operand, against the oracle's FP64 product."""
+    rng = np.random.default_rng(71)
+    M, N, K = 128, 256, 256
+
+    def operand(rows, amax):
+        codes = rng.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+        scales = rng.integers(1, sf_hi + 1, size=(rows, K // 16), dtype=np.uint8)
+        return oracle.Quantized(codes, scales, float(np.float32(amax)), 0)
+
+    qa, qb = operand(M, amax_a), operand(N, amax_b)
+    D = B.gemm(upload_quantized(qa, B), upload_quantized(qb, B), out_dtype=dtype)
+    D_ref, norm = oracle.gemm_ref(qa, qb)
+    assert_gemm_close(D.float().cpu().numpy(), D_ref, norm, bf16=(dtype == torch.bfloat16),
+                      what=f"amax {amax_a:g} x {amax_b:g}")
