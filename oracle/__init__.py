@@ -47,6 +47,14 @@ def lib():
                                    ctypes.c_int, ctypes.c_int, u64, u64, ctypes.c_int, fp,
                                    vp, vp, ctypes.POINTER(fp)]
         L.nvo_quantize.restype = ctypes.c_int
+        L.nvo_quantize_rows.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, u16,
+                                        ctypes.c_int, ctypes.c_int, u64, u64, fp, i64, i64,
+                                        vp, vp]
+        L.nvo_quantize_rows.restype = ctypes.c_int
+        L.nvo_quantize_mt.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, u16,
+                                      ctypes.c_int, ctypes.c_int, u64, u64, ctypes.c_int, fp,
+                                      vp, vp, ctypes.POINTER(fp), ctypes.c_int]
+        L.nvo_quantize_mt.restype = ctypes.c_int
         L.nvo_amax.argtypes = [vp, i64, i64, i64, ctypes.c_int, ctypes.c_int, u16,
                                ctypes.POINTER(fp)]
         L.nvo_amax.restype = ctypes.c_int
@@ -173,22 +181,46 @@ class Quantized:
 
 
 def quantize(x_bf16: np.ndarray, *, transpose=False, rht=False, sign_mask=0, block2d=False,
-             sr=False, seed=0, offset=0, amax=None) -> Quantized:
+             sr=False, seed=0, offset=0, amax=None, threads=1) -> Quantized:
     """Quantize the bf16 matrix ``x_bf16`` (np.uint16 bit patterns, rows x cols) along its
-    rows (or, with ``transpose``, along its columns, i.e. quantize x^T)."""
+    rows (or, with ``transpose``, along its columns, i.e. quantize x^T).  ``threads`` > 1
+    runs the oracle's threaded driver (the same two passes over ranges of rows, same bits)."""
     x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
     rows, cols = x.shape
     R, C = (cols, rows) if transpose else (rows, cols)
     codes = np.zeros((R, C // 2), dtype=np.uint8)
     scales = np.zeros((R, C // 16), dtype=np.uint8)
     amax_out = ctypes.c_float(0.0)
-    st = lib().nvo_quantize(_ptr(x), rows, cols, cols, int(transpose), int(rht), sign_mask,
-                            int(block2d), int(sr), seed, offset, int(amax is not None),
-                            0.0 if amax is None else float(amax), _ptr(codes), _ptr(scales),
-                            ctypes.byref(amax_out))
+    args = (_ptr(x), rows, cols, cols, int(transpose), int(rht), sign_mask, int(block2d),
+            int(sr), seed, offset, int(amax is not None), 0.0 if amax is None else float(amax),
+            _ptr(codes), _ptr(scales), ctypes.byref(amax_out))
+    if threads > 1:
+        st = lib().nvo_quantize_mt(*args, int(threads))
+    else:
+        st = lib().nvo_quantize(*args)
     if st not in (NVO_OK, NVO_ERR_NONFINITE):
         raise ValueError(f"oracle quantize rejected the arguments (status {st})")
     return Quantized(codes, scales, amax_out.value, st)
+
+
+def quantize_rows(x_bf16: np.ndarray, r_begin: int, r_end: int, amax: float, *,
+                  transpose=False, rht=False, sign_mask=0, block2d=False, sr=False, seed=0,
+                  offset=0, out: Quantized = None) -> Quantized:
+    """Quantize only logical rows [r_begin, r_end) of the matrix ``quantize`` would quantize,
+    with the given (whole-tensor) amax, into ``out`` (a full-size Quantized, created if None);
+    the other rows are left as they are.  r_begin is a multiple of 16."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    rows, cols = x.shape
+    R, C = (cols, rows) if transpose else (rows, cols)
+    if out is None:
+        out = Quantized(np.zeros((R, C // 2), dtype=np.uint8),
+                        np.zeros((R, C // 16), dtype=np.uint8), float(amax), NVO_OK)
+    st = lib().nvo_quantize_rows(_ptr(x), rows, cols, cols, int(transpose), int(rht), sign_mask,
+                                 int(block2d), int(sr), seed, offset, float(amax), r_begin,
+                                 r_end, _ptr(out.codes), _ptr(out.scales))
+    if st != NVO_OK:
+        raise ValueError(f"oracle quantize_rows rejected the arguments (status {st})")
+    return out
 
 
 def amax(x_bf16: np.ndarray, *, transpose=False, rht=False, sign_mask=0):

@@ -15,7 +15,7 @@ LIB = os.path.join(HERE, "liboracle.so")
 def build(force: bool = False) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
         return LIB
-    cmd = ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-ffp-contract=off",
+    cmd = ["gcc", "-std=c11", "-O2", "-fPIC", "-shared", "-pthread", "-ffp-contract=off",
            "-fno-fast-math", "-fno-unsafe-math-optimizations", "-o", LIB, SRC, "-lm"]
     subprocess.run(cmd, check=True)
     return LIB

@@ -32,6 +32,7 @@
  */
 #include <float.h>
 #include <math.h>
+#include <pthread.h>
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
@@ -45,7 +46,7 @@ int nvo_version(void) { return 1; }
 /* ------------------------------------------------------------------------------------
  * E2M1 element format.  [P1 Formato NVFP4] 4-bit floating point elements; [MX] E2M1:
  * 1 sign bit, 2 exponent bits (bias 1), 1 mantissa bit.  The eight magnitudes, in code
- * order 0..7, are 0, 0.5, 1, 1.5, 2, 3, 4, 6.  [P2] counts "16 values": 16 bit patterns,
+ * order 0..7, are 0, 0.5, 1, 1.5, 2, 3, 4, 6.  [P2] counts sixteen codes: 16 bit patterns,
  * of which +0 and -0 are the same number.
  * ---------------------------------------------------------------------------------- */
 static const double E2M1_MAGNITUDE[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
@@ -323,62 +324,20 @@ int nvo_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, int tran
     return nonfinite ? NVO_ERR_NONFINITE : NVO_OK;
 }
 
-/* Quantize a bf16 matrix x (rows x cols, row stride ld elements) to NVFP4 along the
- * logical rows of L (see build_rows).
- *
- *   codes  : R' * C' / 2 bytes, row-major, two codes per byte, even column in the low
- *            nibble (READING: the pages fix no packing).
- *   scales : R' * (C' / 16) E4M3 bytes, row-major, one per block of 16 along C'.
- *   amax   : the tensor amax that was used (computed, or `amax_in` if amax_given).
- *
- * block2d: one scale per 16 x 16 tile of L (weights [P1 Escalado 2D]: the same quantized
- * values serve the forward and backward GEMMs); otherwise one per 1 x 16 block [P1
- * Formato NVFP4].  sr: stochastic rounding with element index e = r * C' + c of L.
- * Non-finite data (NaN or Inf anywhere in L): every code and scale is 0, amax is +Inf
- * and the return value is NVO_ERR_NONFINITE (READING). */
-int nvo_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
-                 int transpose, int rht, uint16_t sign_mask, int block2d, int sr,
-                 uint64_t seed, uint64_t offset, int amax_given, float amax_in,
-                 uint8_t* codes, uint8_t* scales, float* amax_out)
+/* Pass 2 of the quantization: block scales and codes of logical rows [r_begin, r_end) of L
+ * (see build_rows), 16 logical rows at a time, with the tensor encode scale s_enc that pass 1
+ * fixed.  r_begin is a multiple of 16, so the strips -- and with block2d the 16 x 16 tiles --
+ * are the same whether the rows are done in one call or in several.  The element index of
+ * stochastic rounding is the absolute e = r * C' + c.  `strip` holds 16 * C' floats. */
+static void quantize_strips(const uint16_t* x, int64_t ld, int transpose, int rht,
+                            uint16_t sign_mask, int block2d, int sr, uint64_t seed,
+                            uint64_t offset, float s_enc, int64_t Rl, int64_t Cl,
+                            int64_t r_begin, int64_t r_end, uint8_t* codes, uint8_t* scales,
+                            float* strip)
 {
-    int64_t Rl = transpose ? cols : rows;
-    int64_t Cl = transpose ? rows : cols;
-    if (Rl <= 0 || Cl <= 0 || (Cl % 16) != 0 || (block2d && (Rl % 16) != 0)) return NVO_ERR_ARG;
     int64_t nb = Cl / 16;
-    memset(codes, 0, (size_t)(Rl * Cl / 2));
-    memset(scales, 0, (size_t)(Rl * nb));
-
-    float* strip = (float*)malloc(sizeof(float) * 16 * (size_t)Cl);
-    if (!strip) return NVO_ERR_ARG;
-
-    /* Pass 1: tensor amax over L (after the transform, when there is one). */
-    float amax = 0.0f;
-    int nonfinite = 0;
-    if (amax_given) {
-        amax = amax_in;
-        if (!(amax >= 0.0f) || isinf(amax)) nonfinite = 1;
-    } else {
-        for (int64_t r0 = 0; r0 < Rl; r0 += 16) {
-            int64_t n = (Rl - r0 < 16) ? (Rl - r0) : 16;
-            build_rows(x, ld, transpose, rht, sign_mask, r0, n, Cl, strip);
-            for (int64_t i = 0; i < n * Cl; ++i) {
-                float a = fabsf(strip[i]);
-                if (!isfinite(a)) nonfinite = 1;
-                else if (a > amax) amax = a;
-            }
-        }
-    }
-    if (nonfinite) {
-        free(strip);
-        *amax_out = INFINITY;
-        return NVO_ERR_NONFINITE;
-    }
-    *amax_out = amax;
-    float s_enc = nvo_tensor_scale(amax);
-
-    /* Pass 2: block scales and codes, 16 logical rows at a time. */
-    for (int64_t r0 = 0; r0 < Rl; r0 += 16) {
-        int64_t n = (Rl - r0 < 16) ? (Rl - r0) : 16;
+    for (int64_t r0 = r_begin; r0 < r_end; r0 += 16) {
+        int64_t n = (r_end - r0 < 16) ? (r_end - r0) : 16;
         build_rows(x, ld, transpose, rht, sign_mask, r0, n, Cl, strip);
         for (int64_t kb = 0; kb < nb; ++kb) {
             float tile_max = 0.0f;
@@ -414,8 +373,218 @@ int nvo_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
             }
         }
     }
+    (void)Rl;
+}
+
+/* Pass 1 over logical rows [r_begin, r_end): the largest finite |value| of L (after the
+ * transform, when there is one) into *amax, and whether any value is NaN or Inf. */
+static int amax_strips(const uint16_t* x, int64_t ld, int transpose, int rht,
+                       uint16_t sign_mask, int64_t Cl, int64_t r_begin, int64_t r_end,
+                       float* amax, float* strip)
+{
+    int nonfinite = 0;
+    float m = 0.0f;
+    for (int64_t r0 = r_begin; r0 < r_end; r0 += 16) {
+        int64_t n = (r_end - r0 < 16) ? (r_end - r0) : 16;
+        build_rows(x, ld, transpose, rht, sign_mask, r0, n, Cl, strip);
+        for (int64_t i = 0; i < n * Cl; ++i) {
+            float a = fabsf(strip[i]);
+            if (!isfinite(a)) nonfinite = 1;
+            else if (a > m) m = a;
+        }
+    }
+    *amax = m;
+    return nonfinite;
+}
+
+/* Quantize a bf16 matrix x (rows x cols, row stride ld elements) to NVFP4 along the
+ * logical rows of L (see build_rows).
+ *
+ *   codes  : R' * C' / 2 bytes, row-major, two codes per byte, even column in the low
+ *            nibble (READING: the pages fix no packing).
+ *   scales : R' * (C' / 16) E4M3 bytes, row-major, one per block of 16 along C'.
+ *   amax   : the tensor amax that was used (computed, or `amax_in` if amax_given).
+ *
+ * block2d: one scale per 16 x 16 tile of L (weights [P1 Escalado 2D]: the same quantized
+ * values serve the forward and backward GEMMs); otherwise one per 1 x 16 block [P1
+ * Formato NVFP4].  sr: stochastic rounding with element index e = r * C' + c of L.
+ * Non-finite data (NaN or Inf anywhere in L): every code and scale is 0, amax is +Inf
+ * and the return value is NVO_ERR_NONFINITE (READING). */
+int nvo_quantize(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                 int transpose, int rht, uint16_t sign_mask, int block2d, int sr,
+                 uint64_t seed, uint64_t offset, int amax_given, float amax_in,
+                 uint8_t* codes, uint8_t* scales, float* amax_out)
+{
+    int64_t Rl = transpose ? cols : rows;
+    int64_t Cl = transpose ? rows : cols;
+    if (Rl <= 0 || Cl <= 0 || (Cl % 16) != 0 || (block2d && (Rl % 16) != 0)) return NVO_ERR_ARG;
+    int64_t nb = Cl / 16;
+    memset(codes, 0, (size_t)(Rl * Cl / 2));
+    memset(scales, 0, (size_t)(Rl * nb));
+
+    float* strip = (float*)malloc(sizeof(float) * 16 * (size_t)Cl);
+    if (!strip) return NVO_ERR_ARG;
+
+    /* Pass 1: tensor amax over L (after the transform, when there is one). */
+    float amax = 0.0f;
+    int nonfinite = 0;
+    if (amax_given) {
+        amax = amax_in;
+        if (!(amax >= 0.0f) || isinf(amax)) nonfinite = 1;
+    } else {
+        nonfinite = amax_strips(x, ld, transpose, rht, sign_mask, Cl, 0, Rl, &amax, strip);
+    }
+    if (nonfinite) {
+        free(strip);
+        *amax_out = INFINITY;
+        return NVO_ERR_NONFINITE;
+    }
+    *amax_out = amax;
+    float s_enc = nvo_tensor_scale(amax);
+
+    /* Pass 2: block scales and codes, 16 logical rows at a time. */
+    quantize_strips(x, ld, transpose, rht, sign_mask, block2d, sr, seed, offset, s_enc, Rl, Cl,
+                    0, Rl, codes, scales, strip);
     free(strip);
     return NVO_OK;
+}
+
+/* Pass 2 alone for logical rows [r_begin, r_end) of L, with a given finite tensor amax (the
+ * whole tensor's, e.g. from nvo_amax): writes only those rows of the full-size codes and scales
+ * arrays.  r_begin must be a multiple of 16 and r_end a multiple of 16 or R'.  Rows quantized
+ * by several such calls equal, bit for bit, one nvo_quantize of the whole tensor with the same
+ * amax: the strips, the tiles and the element indices are the same. */
+int nvo_quantize_rows(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                      int transpose, int rht, uint16_t sign_mask, int block2d, int sr,
+                      uint64_t seed, uint64_t offset, float amax, int64_t r_begin,
+                      int64_t r_end, uint8_t* codes, uint8_t* scales)
+{
+    int64_t Rl = transpose ? cols : rows;
+    int64_t Cl = transpose ? rows : cols;
+    if (Rl <= 0 || Cl <= 0 || (Cl % 16) != 0 || (block2d && (Rl % 16) != 0)) return NVO_ERR_ARG;
+    if (r_begin < 0 || r_begin > r_end || r_end > Rl || r_begin % 16 != 0 ||
+        (r_end % 16 != 0 && r_end != Rl))
+        return NVO_ERR_ARG;
+    if (!(amax >= 0.0f) || isinf(amax)) return NVO_ERR_ARG;
+    int64_t nb = Cl / 16;
+    memset(codes + r_begin * Cl / 2, 0, (size_t)((r_end - r_begin) * Cl / 2));
+    memset(scales + r_begin * nb, 0, (size_t)((r_end - r_begin) * nb));
+    float* strip = (float*)malloc(sizeof(float) * 16 * (size_t)Cl);
+    if (!strip) return NVO_ERR_ARG;
+    quantize_strips(x, ld, transpose, rht, sign_mask, block2d, sr, seed, offset,
+                    nvo_tensor_scale(amax), Rl, Cl, r_begin, r_end, codes, scales, strip);
+    free(strip);
+    return NVO_OK;
+}
+
+/* ------------------------------------------------------------------------------------
+ * A threaded driver of the same two passes, for whole tensors too large for one core in a
+ * test's time and for timing the oracle on all host cores.  The logical rows are cut into
+ * `nthreads` ranges of whole 16-row strips; pass 1 takes each range's maximum and the
+ * largest of them (a maximum does not depend on the order it visits values), pass 2 runs
+ * quantize_strips on each range with the tensor scale of that amax.  Same outputs, bit for
+ * bit, as nvo_quantize.
+ * ---------------------------------------------------------------------------------- */
+typedef struct {
+    const uint16_t* x;
+    int64_t ld, Rl, Cl, r_begin, r_end;
+    int transpose, rht, block2d, sr, pass, nonfinite;
+    uint16_t sign_mask;
+    uint64_t seed, offset;
+    float s_enc, amax;
+    uint8_t* codes;
+    uint8_t* scales;
+} nvo_job;
+
+static void* nvo_job_run(void* arg)
+{
+    nvo_job* j = (nvo_job*)arg;
+    float* strip = (float*)malloc(sizeof(float) * 16 * (size_t)j->Cl);
+    if (!strip) {
+        j->nonfinite = -1;
+        return NULL;
+    }
+    if (j->pass == 1)
+        j->nonfinite = amax_strips(j->x, j->ld, j->transpose, j->rht, j->sign_mask, j->Cl,
+                                   j->r_begin, j->r_end, &j->amax, strip);
+    else
+        quantize_strips(j->x, j->ld, j->transpose, j->rht, j->sign_mask, j->block2d, j->sr,
+                        j->seed, j->offset, j->s_enc, j->Rl, j->Cl, j->r_begin, j->r_end,
+                        j->codes, j->scales, strip);
+    free(strip);
+    return NULL;
+}
+
+static int run_jobs(nvo_job* jobs, int n)
+{
+    pthread_t* t = (pthread_t*)malloc(sizeof(pthread_t) * (size_t)n);
+    if (!t) return -1;
+    int started = 0, failed = 0;
+    for (; started < n; ++started)
+        if (pthread_create(&t[started], NULL, nvo_job_run, &jobs[started]) != 0) break;
+    for (int i = started; i < n; ++i) nvo_job_run(&jobs[i]); /* could not start: run here */
+    for (int i = 0; i < started; ++i) pthread_join(t[i], NULL);
+    for (int i = 0; i < n; ++i)
+        if (jobs[i].nonfinite < 0) failed = 1;
+    free(t);
+    return failed ? -1 : 0;
+}
+
+int nvo_quantize_mt(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
+                    int transpose, int rht, uint16_t sign_mask, int block2d, int sr,
+                    uint64_t seed, uint64_t offset, int amax_given, float amax_in,
+                    uint8_t* codes, uint8_t* scales, float* amax_out, int nthreads)
+{
+    int64_t Rl = transpose ? cols : rows;
+    int64_t Cl = transpose ? rows : cols;
+    if (Rl <= 0 || Cl <= 0 || (Cl % 16) != 0 || (block2d && (Rl % 16) != 0)) return NVO_ERR_ARG;
+    if (nthreads < 1) nthreads = 1;
+    int64_t strips = (Rl + 15) / 16;
+    if (nthreads > strips) nthreads = (int)strips;
+    nvo_job* jobs = (nvo_job*)calloc((size_t)nthreads, sizeof(nvo_job));
+    if (!jobs) return NVO_ERR_ARG;
+    for (int i = 0; i < nthreads; ++i) {
+        nvo_job* j = &jobs[i];
+        j->x = x; j->ld = ld; j->Rl = Rl; j->Cl = Cl;
+        j->r_begin = 16 * (strips * i / nthreads);
+        j->r_end = 16 * (strips * (i + 1) / nthreads);
+        if (j->r_end > Rl) j->r_end = Rl;
+        j->transpose = transpose; j->rht = rht; j->block2d = block2d; j->sr = sr;
+        j->sign_mask = sign_mask; j->seed = seed; j->offset = offset;
+        j->codes = codes; j->scales = scales;
+    }
+    memset(codes, 0, (size_t)(Rl * Cl / 2));
+    memset(scales, 0, (size_t)(Rl * (Cl / 16)));
+    float amax = 0.0f;
+    int nonfinite = 0;
+    if (amax_given) {
+        amax = amax_in;
+        if (!(amax >= 0.0f) || isinf(amax)) nonfinite = 1;
+    } else {
+        for (int i = 0; i < nthreads; ++i) jobs[i].pass = 1;
+        if (run_jobs(jobs, nthreads) != 0) {
+            free(jobs);
+            return NVO_ERR_ARG;
+        }
+        for (int i = 0; i < nthreads; ++i) {
+            if (jobs[i].nonfinite) nonfinite = 1;
+            if (jobs[i].amax > amax) amax = jobs[i].amax;
+        }
+    }
+    if (nonfinite) {
+        free(jobs);
+        *amax_out = INFINITY;
+        return NVO_ERR_NONFINITE;
+    }
+    *amax_out = amax;
+    for (int i = 0; i < nthreads; ++i) {
+        jobs[i].pass = 2;
+        jobs[i].nonfinite = 0;
+        jobs[i].s_enc = nvo_tensor_scale(amax);
+    }
+    int rc = run_jobs(jobs, nthreads);
+    free(jobs);
+    return rc == 0 ? NVO_OK : NVO_ERR_ARG;
 }
 
 /* ------------------------------------------------------------------------------------

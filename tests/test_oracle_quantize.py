@@ -235,3 +235,51 @@ def test_per_element_error_bound(sr):
     assert np.all(err <= allowed * (1 + 1e-6) + 1e-30)
     # e4m3 block scales keep every block max within one E4M3 rounding of 6 units
     assert np.all(sat <= np.abs(xf) * 2.0 ** -4 + 1e-30)
+
+
+_SPLIT_MODES = [
+    dict(),
+    dict(sr=True, seed=3, offset=2),
+    dict(block2d=True),
+    dict(transpose=True, block2d=True),
+    dict(transpose=True, rht=True, sign_mask=0x1234, sr=True, seed=9, offset=1),
+    dict(transpose=True, rht=True, sign_mask=0xBEEF),
+]
+
+
+@pytest.mark.parametrize("kw", _SPLIT_MODES)
+@pytest.mark.parametrize("shape", [(512, 768), (48, 320)])
+def test_row_ranges_and_threads_give_the_whole_call(kw, shape):
+    """The element index of stochastic rounding is the absolute row's (e = r * C' + c), and a
+    16 x 16 tile never straddles two calls, so quantizing the logical rows in several ranges
+    with the whole tensor's amax -- or with the threaded driver -- gives the whole call's bits."""
+    x = synth.gradients(shape, seed=11)
+    whole = oracle.quantize(x, **kw)
+    R = whole.rows
+    cuts = [0, 16, 16 * max(1, R // 48), R]
+    out = None
+    for r0, r1 in zip(cuts[:-1], cuts[1:]):
+        if r1 > r0:
+            out = oracle.quantize_rows(x, r0, r1, whole.amax, out=out, **kw)
+    assert np.array_equal(out.codes, whole.codes) and np.array_equal(out.scales, whole.scales)
+    for threads in (2, 5, 64):
+        mt = oracle.quantize(x, threads=threads, **kw)
+        assert mt.amax == whole.amax and mt.status == whole.status
+        assert np.array_equal(mt.codes, whole.codes)
+        assert np.array_equal(mt.scales, whole.scales)
+
+
+def test_row_ranges_reject_misaligned_starts_and_bad_amax():
+    x = synth.activations((64, 64), seed=1)
+    with pytest.raises(ValueError):
+        oracle.quantize_rows(x, 8, 64, 1.0)
+    with pytest.raises(ValueError):
+        oracle.quantize_rows(x, 0, 64, float("inf"))
+
+
+def test_threaded_driver_flags_non_finite_input():
+    x = synth.activations((256, 256), seed=2)
+    x[200, 7] = 0x7FC0  # NaN
+    q = oracle.quantize(x, threads=4)
+    assert q.status == oracle.NVO_ERR_NONFINITE and np.isinf(q.amax)
+    assert not q.codes.any() and not q.scales.any()
