@@ -33,6 +33,26 @@ class Operand(ctypes.Structure):
 
 
 _lib = None
+_poison = False
+
+
+def set_output_poisoning(enabled: bool):
+    """Debug aid for tests: when enabled, every output buffer this module allocates is first
+    filled with a pattern no kernel writes (codes and scales 0xFF bytes, FP32 / bf16 results and
+    amax NaN; workspaces 0xFF bytes), so that a kernel that leaves part of its output unwritten,
+    or reads scratch it did not write, cannot pass a check by finding an earlier, identical
+    result in recycled memory."""
+    global _poison
+    _poison = bool(enabled)
+
+
+def _poisoned(t):
+    if _poison:
+        if t.dtype == torch.uint8:
+            t.fill_(0xFF)
+        else:
+            t.fill_(float("nan"))
+    return t
 
 
 def lib():
@@ -149,9 +169,10 @@ class QuantizedTensor:
 
     def __init__(self, rows, cols, device="cuda"):
         self.rows, self.cols = rows, cols
-        self.codes = torch.empty((rows, cols // 2), dtype=torch.uint8, device=device)
-        self.scales = torch.empty((scales_bytes(rows, cols),), dtype=torch.uint8, device=device)
-        self.amax = torch.zeros((1,), dtype=torch.float32, device=device)
+        self.codes = _poisoned(torch.empty((rows, cols // 2), dtype=torch.uint8, device=device))
+        self.scales = _poisoned(torch.empty((scales_bytes(rows, cols),), dtype=torch.uint8,
+                                            device=device))
+        self.amax = _poisoned(torch.zeros((1,), dtype=torch.float32, device=device))
 
     def operand(self):
         return Operand(self.codes.data_ptr(), self.scales.data_ptr(), self.amax.data_ptr(),
@@ -169,7 +190,7 @@ def _dtype_code(dtype):
 def _workspace(nbytes, device):
     if nbytes == 0:
         return None
-    return torch.empty((nbytes,), dtype=torch.uint8, device=device)
+    return _poisoned(torch.empty((nbytes,), dtype=torch.uint8, device=device))
 
 
 def quantize(x, flags, seed=0, offset=0, out_row=None, out_col=None, workspace=None,
@@ -243,7 +264,7 @@ def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None, 
     type is out.dtype when `out` is given, else `out_dtype`."""
     name = "nvfp4_gemm_mx" if mx else "nvfp4_gemm"
     if out is None:
-        out = torch.empty((A.rows, B.rows), dtype=out_dtype, device=A.codes.device)
+        out = _poisoned(torch.empty((A.rows, B.rows), dtype=out_dtype, device=A.codes.device))
     _check_out(out, A.rows, B.rows, name)
     d_dtype = _dtype_code(out.dtype)
     oa, ob = A.operand(), B.operand()
@@ -256,11 +277,12 @@ def gemm(A, B, out=None, out_dtype=torch.float32, dev_status=None, stream=None, 
 def gemm_amax(A, B, sign_mask, out=None, amax_out=None, dev_status=None, stream=None):
     """nvfp4_gemm_amax: bf16 D = A . B^T plus amax_out = [max |D|, max |RHT(D)|] (FP32)."""
     if out is None:
-        out = torch.empty((A.rows, B.rows), dtype=torch.bfloat16, device=A.codes.device)
+        out = _poisoned(torch.empty((A.rows, B.rows), dtype=torch.bfloat16,
+                                    device=A.codes.device))
     _check_out(out, A.rows, B.rows, "nvfp4_gemm_amax")
     assert out.dtype == torch.bfloat16
     if amax_out is None:
-        amax_out = torch.empty(2, dtype=torch.float32, device=A.codes.device)
+        amax_out = _poisoned(torch.empty(2, dtype=torch.float32, device=A.codes.device))
     oa, ob = A.operand(), B.operand()
     st = lib().nvfp4_gemm_amax(ctypes.byref(oa), ctypes.byref(ob), _ptr(out), out.stride(0),
                                sign_mask, _ptr(amax_out), _ptr(dev_status), _stream(stream))
@@ -280,7 +302,7 @@ def linear_fprop(X, W, out=None, out_dtype=torch.float32, workspace=None, dev_st
     T, I = X.shape
     O = W.shape[0]
     if out is None:
-        out = torch.empty((T, O), dtype=out_dtype, device=X.device)
+        out = _poisoned(torch.empty((T, O), dtype=out_dtype, device=X.device))
     _check_out(out, T, O, "nvfp4_linear_fprop")
     if workspace is None:
         workspace = _workspace(linear_workspace_bytes(T, I, O), X.device)
@@ -295,7 +317,7 @@ def linear_dgrad(dY, W, seed, offset, out=None, out_dtype=torch.float32, workspa
     T, O = dY.shape
     I = W.shape[1]
     if out is None:
-        out = torch.empty((T, I), dtype=out_dtype, device=dY.device)
+        out = _poisoned(torch.empty((T, I), dtype=out_dtype, device=dY.device))
     _check_out(out, T, I, "nvfp4_linear_dgrad")
     if workspace is None:
         workspace = _workspace(linear_workspace_bytes(T, I, O), dY.device)
@@ -314,7 +336,7 @@ def linear_dgrad_quantized(dY, W, seed, offset, sign_mask, next_seed, next_offse
     T, O = dY.shape
     I = W.shape[1]
     if out is None:
-        out = torch.empty((T, I), dtype=torch.bfloat16, device=dY.device)
+        out = _poisoned(torch.empty((T, I), dtype=torch.bfloat16, device=dY.device))
     _check_out(out, T, I, "nvfp4_linear_dgrad_quantized")
     if out.dtype != torch.bfloat16:
         raise TypeError("nvfp4_linear_dgrad_quantized: dX must be bfloat16")
@@ -338,7 +360,7 @@ def linear_wgrad(dY, X, sign_mask, seed, offset, out=None, out_dtype=torch.float
     T, O = dY.shape
     I = X.shape[1]
     if out is None:
-        out = torch.empty((O, I), dtype=out_dtype, device=dY.device)
+        out = _poisoned(torch.empty((O, I), dtype=out_dtype, device=dY.device))
     _check_out(out, O, I, "nvfp4_linear_wgrad")
     if workspace is None:
         workspace = _workspace(linear_workspace_bytes(T, I, O), dY.device)

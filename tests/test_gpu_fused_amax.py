@@ -1,13 +1,15 @@
 """nvfp4_gemm_amax: a bf16 GEMM that also emits the maxima the next quantization of its output
 needs (max |D| and max |RHT(D)| along the rows), so that quantization can skip its amax pass.
 
-D is a GPU result, so no oracle value is derived from it; the checks are properties that hold
-at any size:
-* D is bit-identical to nvfp4_gemm's bf16 output and matches the oracle's FP64 product within
-  the usual tolerance;
-* the fused maxima equal, bit for bit, the ones the quantizer's own amax pass computes on D;
+D is the GEMM's own output (FP32 accumulation in an order the oracle does not reproduce), so it
+is checked against the oracle's FP64 product within the usual tolerance; every quantity derived
+from D -- its two maxima, its quantized operands -- is a function of D's bits, so the oracle
+computes the expected value of each from those same bits:
+* D is bit-identical to nvfp4_gemm's bf16 output and matches the oracle's FP64 product;
+* the fused maxima equal, bit for bit, the oracle's amax of D and of its random Hadamard
+  transform along the rows (and the quantizer's own amax pass on D);
 * quantizing D with the fused maxima (NVFP4_AMAX_GIVEN) gives exactly the codes, scales and
-  amax of the quantization that runs its amax pass."""
+  amax of the quantization that runs its amax pass, and of the oracle's quantization of D."""
 import ctypes
 
 import numpy as np
@@ -16,7 +18,7 @@ import torch
 
 import oracle
 import synth
-from nvfp4_testlib import assert_gemm_close, need_gpu, to_device_bf16
+from nvfp4_testlib import assert_gemm_close, assert_quantized_equal, need_gpu, to_device_bf16
 
 nv = pytest.importorskip("nvfp4_bit_quantized_03_b200")
 B = nv.binding
@@ -51,6 +53,13 @@ def test_fused_maxima_equal_the_quantizers_amax(M, N, K):
     got = amax.cpu().numpy().view(np.uint32)
     want = np.array([qr.amax.item(), qc.amax.item()], dtype=np.float32).view(np.uint32)
     assert np.array_equal(got, want), (got, want)
+    # the oracle's maxima of the same bf16 bits: max |D| and max |RHT(D)| with 16-row blocks
+    D_bits = D.view(torch.int16).cpu().numpy().view(np.uint16)
+    plain, st0 = oracle.amax(D_bits)
+    rht, st1 = oracle.amax(D_bits, transpose=True, rht=True, sign_mask=mask)
+    assert st0 == 0 and st1 == 0
+    want_oracle = np.array([plain, rht], dtype=np.float32).view(np.uint32)
+    assert np.array_equal(got, want_oracle), (got, want_oracle)
 
 
 @pytest.mark.parametrize("sr", [False, True])
@@ -99,6 +108,13 @@ def test_dgrad_quantized_equals_the_unfused_sequence(T, I, O):
         assert torch.equal(got.amax, want.amax)
     D_ref, norm = oracle.gemm_ref(*oracle.dgrad_operands(dY, W, 3, 1))
     assert_gemm_close(dX.float().cpu().numpy(), D_ref, norm, bf16=True, what="dgrad_quantized dX")
+    # dX's operands against the oracle's quantization of dX's bits: row-wise SR on stream
+    # next_offset, RHT'd column-wise SR on stream next_offset + 1
+    dX_bits = dX.view(torch.int16).cpu().numpy().view(np.uint16)
+    assert_quantized_equal(qr, oracle.quantize(dX_bits, sr=True, seed=11, offset=5), "dX row")
+    assert_quantized_equal(qc, oracle.quantize(dX_bits, transpose=True, rht=True,
+                                               sign_mask=mask, sr=True, seed=11, offset=6),
+                           "dX col")
 
 
 def test_dgrad_quantized_rejects_bad_operands():

@@ -68,48 +68,3 @@ def test_fprop_small_workload():
 def test_one_layer_4096_full():
     wl = synth.layer_4096()
     _run_layer(wl.linears[0], wl.seed)
-
-
-def _sample(n, k=96, seed=0):
-    rng = np.random.default_rng(seed + n)
-    return np.sort(rng.choice(n, size=min(k, n), replace=False))
-
-
-def _check_workload_linear(wl, which):
-    """fprop, dgrad and wgrad of one linear of a workload through the C ABI against the
-    oracle: 96 sampled rows x all columns and all rows x 96 sampled columns of each GEMM."""
-    lin = {l.name: l for l in wl.linears}[which]
-    idx = [l.name for l in wl.linears].index(which)
-    X, W, dY = synth.linear_inputs(lin, wl.seed, layer_index=idx)
-    mask = oracle.sign_mask_from_seed(wl.seed)
-    Xd, Wd, dYd = to_device_bf16(X), to_device_bf16(W), to_device_bf16(dY)
-    outs = {"fprop": B.linear_fprop(Xd, Wd),
-            "dgrad": B.linear_dgrad(dYd, Wd, wl.seed, 0),
-            "wgrad": B.linear_wgrad(dYd, Xd, mask, wl.seed, 0)}
-    ops = {"fprop": oracle.fprop_operands(X, W),
-           "dgrad": oracle.dgrad_operands(dY, W, wl.seed, 0),
-           "wgrad": oracle.wgrad_operands(dY, X, mask, wl.seed, 0)}
-    for name, D in outs.items():
-        qa, qb = ops[name]
-        r, c = _sample(qa.rows), _sample(qb.rows, seed=1)
-        Dr, nr = oracle.gemm_ref(qa, qb, rows=r)
-        assert_gemm_close(D[torch.from_numpy(r).cuda()].cpu().numpy(), Dr, nr, what=name + " rows")
-        Dc, nc = oracle.gemm_ref(qa, qb, cols=c)
-        assert_gemm_close(D[:, torch.from_numpy(c).cuda()].cpu().numpy(), Dc, nc,
-                          what=name + " cols")
-
-
-@pytest.mark.slow
-@pytest.mark.parametrize("which", ["up", "down"])
-def test_mlp_12b_sampled(which):
-    """12B-class MLP shapes (tokens 8192, 5120 <-> 20480), the shapes the benchmark times."""
-    _check_workload_linear(synth.mlp_12b(), which)
-
-
-@pytest.mark.slow
-@pytest.mark.parametrize("which", ["qkv", "o", "down"])
-def test_dense_8b_layer_sampled(which):
-    """8B-class dense layer at tokens 16384, d 4096: QKV 4096 -> 6144, O 4096 -> 4096 and the
-    MLP down-projection 14336 -> 4096 (gate and up share the down-projection's sizes
-    transposed, which the 12B-class case already covers at other sizes)."""
-    _check_workload_linear(synth.dense_8b_layer(), which)
