@@ -317,11 +317,15 @@ nvfp4_status nvfp4_linear_dgrad_quantized(const void* dY, const void* W, int64_t
  * Same arguments, rules and results as nvfp4_quantize, minus `workspace`: the partial maxima
  * of the amax pass live in a file-scope device array of NVFP4_NOALLOC_MAX_PARTIALS 32-bit slots
  * (8 KB per GPU that loads the library, held until the process exits).  The call allocates
- * nothing.  The first call on each device looks up the array's address; make it before any
- * stream capture begins.  Calls share the array: calls whose kernels overlap on the GPU
- * (several streams or host threads on one device) race and may give wrong results; calls on
- * one stream are safe.  A shape needing more slots than the array holds returns
- * NVFP4_ERR_SHAPE.
+ * nothing.  The first call on each device looks up the array's address and keeps it for the
+ * life of the process; make that first call before any stream capture begins, and do not use
+ * this entry point across a cudaDeviceReset (the kept address would belong to the destroyed
+ * context).  Calls share the array: calls whose kernels overlap on the GPU (several streams or
+ * host threads on one device) race and may give wrong results; calls queued on one stream are
+ * ordered and safe.  A call whose amax pass would use more CTAs than the array has slots
+ * returns NVFP4_ERR_SHAPE; the amax pass never launches more than 2048 CTAs, so no shape that
+ * nvfp4_quantize accepts is rejected for this reason.  With NVFP4_AMAX_GIVEN there is no amax
+ * pass and the array is not touched.
  */
 #define NVFP4_NOALLOC_MAX_PARTIALS 2048
 nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows, int64_t cols, int64_t ld,

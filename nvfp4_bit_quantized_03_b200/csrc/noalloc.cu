@@ -10,14 +10,15 @@
 //
 // The scratch is NVFP4_NOALLOC_MAX_PARTIALS (2048) 32-bit slots, 8 KB; every GPU that loads
 // the library holds it until the process exits.  The first call on each device looks up the
-// array's device address (cudaGetSymbolAddress); make that first call before any stream
-// capture begins.  All calls share the array: two calls whose kernels overlap on the GPU
-// (different streams, or different host threads on one device) race on it and may produce
-// wrong results; calls queued on one stream are ordered and safe.  Nothing in it has to start
-// at zero: each call's amax pass writes every slot that call's quantize pass reads.  A call
-// whose amax pass would need more slots than the array holds is rejected with
-// NVFP4_ERR_SHAPE (the amax pass of this library uses at most 2048 CTAs, so every shape
-// nvfp4_quantize accepts fits).
+// array's device address (cudaGetSymbolAddress) and keeps it; make that first call before
+// any stream capture begins, and do not call this entry point across a cudaDeviceReset, which
+// destroys the context the kept address belongs to.  All calls share the array: two calls
+// whose kernels overlap on the GPU (different streams, or different host threads on one
+// device) race on it and may produce wrong results; calls queued on one stream are ordered and
+// safe.  Nothing in it has to start at zero: each call's amax pass writes every slot that
+// call's quantize pass reads.  A call whose amax pass would launch more CTAs than the array
+// has slots is rejected with NVFP4_ERR_SHAPE; the amax pass caps its grid at 2048 CTAs, so the
+// check only guards that invariant and no shape nvfp4_quantize accepts fails it.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -65,13 +66,17 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x_bf16, int64_t rows,
                                                const nvfp4_operand* out_col, int* dev_status,
                                                void* stream)
 {
-    // nvfp4_quantize keeps one set of amax partials (nvfp4_workspace_bytes also covers the
-    // dual mode's second set, which this entry point never runs).
-    const size_t need =
-        (flags & NVFP4_AMAX_GIVEN) ? 0 : sizeof(uint32_t) * static_cast<size_t>(nvfp4::kMaxPartials);
-    if (need > sizeof(uint32_t) * kScratchSlots) return NVFP4_ERR_SHAPE;
+    // nvfp4_quantize runs the plain amax pass (one partial maximum per CTA) unless the caller
+    // gives the amax; the pass's grid for this shape on this device must fit the array.
     uint32_t* scratch = nullptr;
-    if (need > 0) {
+    if (!(flags & NVFP4_AMAX_GIVEN)) {
+        if (rows > 0 && cols > 0) {
+            int dev = 0, sms = 0;
+            if (cudaGetDevice(&dev) != cudaSuccess ||
+                cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+                return NVFP4_ERR_CUDA;
+            if (nvfp4::amax_grid(rows, cols, false, sms) > kScratchSlots) return NVFP4_ERR_SHAPE;
+        }
         const nvfp4_status st = scratch_address(&scratch);
         if (st != NVFP4_OK) return st;
     }

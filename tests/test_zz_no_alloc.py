@@ -67,6 +67,53 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
             assert _same(got_c, want_c), f"column-wise output differs for {shape}"
 
 
+def test_noalloc_two_calls_queued_on_one_stream_without_a_sync():
+    """Calls queued back to back on one stream are ordered: the second call's amax pass
+    overwrites the scratch slots only after the first call's quantize pass has read them."""
+    need_gpu()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cases = [((8192, 4096), B.ROWWISE | B.SR, synth.gradients, 21),
+             ((2048, 1024), B.ROWWISE | B.COLWISE, synth.activations, 22)]
+    got = []
+    for shape, flags, gen, seed in cases:
+        x = to_device_bf16(gen(shape, seed=seed))
+        rows, cols = shape
+        r = B.QuantizedTensor(rows, cols) if flags & B.ROWWISE else None
+        c = B.QuantizedTensor(cols, rows) if flags & B.COLWISE else None
+        st = _call_noalloc(x, flags, seed, 1, r, c, status)
+        assert st == B.OK, B.lib().nvfp4_status_string(st)
+        got.append((x, flags, seed, r, c))
+    for x, flags, seed, r, c in got:
+        want_r, want_c = B.quantize(x, flags, seed=seed, offset=1)
+        if r is not None:
+            assert _same(r, want_r)
+        if c is not None:
+            assert _same(c, want_c)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
+def test_noalloc_amax_given_and_mx():
+    """NVFP4_AMAX_GIVEN (no amax pass, the scratch is not touched) and the MXFP4 flag through
+    this entry point, against nvfp4_quantize with the same flags."""
+    need_gpu()
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    x = to_device_bf16(synth.activations((1024, 2048), seed=23))
+    want_r, _ = B.quantize(x, B.ROWWISE)
+    got_r = B.QuantizedTensor(1024, 2048)
+    got_r.amax.copy_(want_r.amax)
+    st = _call_noalloc(x, B.ROWWISE | B.AMAX_GIVEN, 0, 0, got_r, None, status)
+    assert st == B.OK
+    assert _same(got_r, want_r)
+    flags = B.ROWWISE | B.COLWISE | B.MX
+    got_r, got_c = B.QuantizedTensor(1024, 2048), B.QuantizedTensor(2048, 1024)
+    assert _call_noalloc(x, flags, 0, 0, got_r, got_c, status) == B.OK
+    want_r, want_c = B.quantize(x, flags)
+    assert _same(got_r, want_r) and _same(got_c, want_c)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+
 def test_noalloc_rejects_bad_arguments_like_the_workspace_entry_point():
     need_gpu()
     out = B.QuantizedTensor(256, 512)
