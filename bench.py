@@ -79,43 +79,103 @@ def whole_job_rate(units_per_rank: float, world: int, seconds_max: float) -> flo
 # ---- clocks ------------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi (every 50 ms) while running.
+    """Samples the SM clock, power and the clock-event (throttle) reasons of one GPU while
+    running: through NVML every 2 ms (read-only queries), else with nvidia-smi every 50 ms.
     `mark()` opens and closes the window whose samples `summary()` reports."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, uuid: str = None, period_s: float = 0.002):
         self.device_index = device_index
+        self.uuid = uuid
+        self.period_s = period_s
         self.proc = None
-        self.samples = []  # (host time, csv line)
+        self.nvml = None
+        self.samples = []  # (host time, sm MHz, max MHz, watts, set of active reasons)
         self.thread = None
+        self.stop = threading.Event()
         self.window = [None, None]
+        self.source = None
 
     def __enter__(self):
+        if not self._start_nvml():
+            self._start_smi()
+        return self
+
+    def _start_nvml(self):
+        try:
+            import pynvml as N
+            N.nvmlInit()
+            h = None
+            if self.uuid:
+                try:
+                    h = N.nvmlDeviceGetHandleByUUID(self.uuid)
+                except N.NVMLError:
+                    h = None
+            if h is None:
+                h = N.nvmlDeviceGetHandleByIndex(self.device_index)
+            bits = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap}
+            smax = N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM)
+        except Exception:
+            return False
+        self.nvml = N
+        self.source = "nvml"
+
+        def poll():
+            while not self.stop.is_set():
+                try:
+                    sm = N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM)
+                    watts = N.nvmlDeviceGetPowerUsage(h) / 1000.0
+                    active = N.nvmlDeviceGetCurrentClocksEventReasons(h)
+                    reasons = {k for k, b in bits.items() if active & b}
+                    self.samples.append((time.time(), float(sm), float(smax), watts, reasons))
+                except Exception:
+                    pass
+                self.stop.wait(self.period_s)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        return True
+
+    def _start_smi(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.device_index), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.source = "nvidia-smi"
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
             t0 = time.time()
             while not self.samples and time.time() - t0 < 10 and self.proc.poll() is None:
                 time.sleep(0.05)  # the first sample marks nvidia-smi as running
         except OSError:
             self.proc = None
-        return self
 
-    def _read(self):
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.samples.append((time.time(), line.strip()))
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm, smax, watts = float(parts[0]), float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            reasons = {n for n, v in zip(self.REASONS, parts[3:7])
+                       if v.lower().startswith("active")}
+            self.samples.append((time.time(), sm, smax, watts, reasons))
 
     def mark(self, which):
         self.window[0 if which == "start" else 1] = time.time()
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             time.sleep(0.1)
             self.proc.terminate()
@@ -123,32 +183,26 @@ class ClockSampler:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-            if self.thread is not None:
-                self.thread.join(timeout=2)
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+        if self.nvml is not None:
+            try:
+                self.nvml.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self):
         t0, t1 = self.window
-        lines = [l for t, l in self.samples
-                 if (t0 is None or t >= t0) and (t1 is None or t <= t1 + 0.05)]
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 7:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                smax.append(float(parts[1]))
-                power.append(float(parts[2]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[3:7]):
-                if val.lower().startswith("active"):
-                    reasons.add(name)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "power_w_max": max(power), "reasons": sorted(reasons), "samples": len(sm)}
+        rows = [r for r in list(self.samples)
+                if (t0 is None or r[0] >= t0) and (t1 is None or r[0] <= t1 + 0.002)]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
+        reasons = set().union(*[r[4] for r in rows])
+        return {"sm_mhz": statistics.median(r[1] for r in rows),
+                "sm_max_mhz": max(r[2] for r in rows),
+                "power_w_max": max(r[3] for r in rows), "reasons": sorted(reasons),
+                "samples": len(rows), "source": self.source}
 
 
 # ---- the workload ------------------------------------------------------------------------
@@ -281,43 +335,114 @@ class Step:
 
 # ---- CPU oracle leg ----------------------------------------------------------------------
 
-def oracle_sample(workload, tokens=128, max_out=512, max_in=4096):
+def host_threads(cap=64):
+    """Host cores this process may run on."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    return max(1, min(cap, n))
+
+
+def blas_threads():
+    """Threads numpy's BLAS uses for the FP64 reference products (1 if it cannot be told)."""
+    try:
+        from threadpoolctl import threadpool_info
+        return max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    except Exception:
+        return 1
+
+
+def oracle_sample(workload, tokens=128, max_out=512, max_in=4096, threads=1):
     """Time the CPU oracle on a bounded sample of the workload: for every linear, a
     `tokens` x min(I, max_in) activation, a min(O, max_out) x min(I, max_in) weight and a
     `tokens` x min(O, max_out) gradient drawn with the workload's generators and seed; the
-    timed part is the three GEMMs' operand quantizations and FP64 reference products.
-    Returns (seconds, GEMM flops of the sample, threads used)."""
+    timed part is the three GEMMs' operand quantizations (the C oracle on `threads` threads)
+    and their FP64 reference products (numpy matmul).
+    Returns (seconds, GEMM flops of the sample)."""
     import oracle
     inputs = []
     for li, lin in enumerate(workload.linears):
         small = synth.Linear(lin.name, tokens, min(lin.I, max_in), min(lin.O, max_out))
         inputs.append(synth.linear_inputs(small, workload.seed, layer_index=li))
     mask = oracle.sign_mask_from_seed(workload.seed)
+    s = workload.seed
     flops = 0
     t0 = time.perf_counter()
     for X, W, dY in inputs:
-        for qa, qb in (oracle.fprop_operands(X, W),
-                       oracle.dgrad_operands(dY, W, workload.seed, 0),
-                       oracle.wgrad_operands(dY, X, mask, workload.seed, 0)):
+        q = dict(threads=threads)
+        for qa, qb in ((oracle.quantize(X, **q), oracle.quantize(W, block2d=True, **q)),
+                       (oracle.quantize(dY, sr=True, seed=s, offset=0, **q),
+                        oracle.quantize(W, transpose=True, block2d=True, **q)),
+                       (oracle.quantize(dY, transpose=True, rht=True, sign_mask=mask, sr=True,
+                                        seed=s, offset=1, **q),
+                        oracle.quantize(X, transpose=True, rht=True, sign_mask=mask, **q))):
             oracle.gemm_ref(qa, qb)
             flops += 2 * qa.rows * qb.rows * qa.cols
-    secs = time.perf_counter() - t0
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    except Exception:
-        threads = 1
-    return secs, flops, threads
+    return time.perf_counter() - t0, flops
+
+
+# The quantizer sweep's modes for the CPU baseline: (name, oracle calls, outputs).  Bytes are
+# counted as for the GPU: two 2-byte reads of every element (amax pass, quantize pass) plus
+# 0.5 B of codes and 1/16 B of scales per element per output.
+CPU_QUANT_MODES = (
+    ("1x16_rtn_row", ({},), 1),
+    ("16x16_2d_rowcol", ({"block2d": True}, {"block2d": True, "transpose": True}), 2),
+    ("1x16_sr_row", ({"sr": True, "seed": 1},), 1),
+    ("rht_1x16_sr_col", ({"transpose": True, "rht": True, "sign_mask": 0x5A3C, "sr": True,
+                          "seed": 1},), 1),
+)
+
+
+def cpu_quantize_baseline(threads, log2n_1t=(20, 22, 24), log2n_all=(20, 22, 24, 26)):
+    """The oracle's quantizer in GB/s of algorithmic bytes on tensors of the quantizer sweep
+    (2^n bf16 elements in rows of 4096, N(0,1) with 1 % x50 outliers), single-threaded and on
+    `threads` threads.  Per mode the rate at the largest size is reported; sizes above those
+    timed are not run (the CPU rate does not depend on the size once the tensor is out of
+    cache)."""
+    import oracle
+    out = {}
+    for label, sizes, th in (("1t", log2n_1t, 1), ("all", log2n_all, threads)):
+        per_mode = {}
+        for log2n in sizes:
+            rows, cols = synth.quant_sweep_shape(log2n)
+            x = synth.activations((rows, cols), seed=synth.QUANT_SWEEP_SEED)
+            n = rows * cols
+            for name, calls, outs in CPU_QUANT_MODES:
+                t0 = time.perf_counter()
+                for kw in calls:
+                    oracle.quantize(x, threads=th, **kw)
+                secs = time.perf_counter() - t0
+                per_mode[name] = n * (4 + outs * (0.5 + 1 / 16)) / secs / 1e9
+            del x
+        total_bytes = sum(4 + outs * (0.5 + 1 / 16) for _, _, outs in CPU_QUANT_MODES)
+        # the modes' aggregate: all four modes' bytes over their summed time, per element
+        agg = total_bytes / sum((4 + outs * (0.5 + 1 / 16)) / per_mode[name]
+                                for name, _, outs in CPU_QUANT_MODES)
+        out[label] = {"gbps": agg, "threads": th, "log2n": max(sizes), "modes": per_mode}
+    return {"value": out["all"]["gbps"], "unit": "GB/s", "cores": threads,
+            "value_single_thread": out["1t"]["gbps"],
+            "kind": "oracle",
+            "sample": "quantizer sweep tensors 2^n bf16 elements in rows of 4096 (N(0,1), 1% x50): "
+                      f"single thread up to 2^{max(log2n_1t)}, {threads} threads up to "
+                      f"2^{max(log2n_all)}; modes 1x16 RTN row, 16x16 2D row+col, 1x16 SR row, "
+                      "RHT+1x16 SR col; 4.5625 B/elem per one-output call, 5.125 for row+col; "
+                      "larger sweep sizes not run",
+            "single_thread": out["1t"], "all_cores": out["all"]}
 
 
 def cpu_baseline(workload):
-    secs, flops, threads = oracle_sample(workload, tokens=1024, max_out=2048, max_in=5120)
+    threads = host_threads()
+    secs, flops = oracle_sample(workload, tokens=1024, max_out=2048, max_in=5120,
+                                threads=threads)
     return {"value": flops / secs / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "oracle_threads": threads, "blas_threads": blas_threads(),
             "sample": "per linear: 1024 tokens x min(O,2048) out- x min(I,5120) in-features drawn "
                       "with the workload's generators; fprop/dgrad/wgrad operand quantization "
-                      "(C oracle, 1 thread) + FP64 reference GEMMs (numpy matmul of the "
-                      "dequantized operands)",
-            "seconds": secs}
+                      f"(C oracle, {threads} threads) + FP64 reference GEMMs (numpy matmul of "
+                      "the dequantized operands)",
+            "seconds": secs,
+            "quantize": cpu_quantize_baseline(threads)}
 
 
 def run_reference(args):
@@ -325,17 +450,18 @@ def run_reference(args):
     if rank != 0:
         return 0
     wl = synth.mlp_12b()
+    threads = host_threads()
     for _ in range(args.warmup):
-        oracle_sample(wl, tokens=128, max_out=512, max_in=4096)
-    times, flops, threads = [], 0, 1
+        oracle_sample(wl, tokens=128, max_out=512, max_in=4096, threads=threads)
+    times, flops = [], 0
     for _ in range(args.steps):
-        secs, flops, threads = oracle_sample(wl, tokens=128, max_out=512, max_in=4096)
+        secs, flops = oracle_sample(wl, tokens=128, max_out=512, max_in=4096, threads=threads)
         times.append(secs)
     total = sum(times)
     value = flops * len(times) / total / 1e12
     sample = ("per linear: 128 tokens x min(O,512) out- x min(I,4096) in-features drawn with "
-              "the workload's generators; operand quantization (C oracle, 1 thread) + FP64 "
-              "reference GEMMs (numpy matmul)")
+              f"the workload's generators; operand quantization (C oracle, {threads} threads) + "
+              "FP64 reference GEMMs (numpy matmul)")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
@@ -369,7 +495,10 @@ def run_ours(args):
             dist.barrier()
 
     events = {"gemm": [], "quant": []}
-    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+    props = torch.cuda.get_device_properties(device)
+    uuid = getattr(props, "uuid", None)
+    uuid = f"GPU-{uuid}" if uuid is not None and not str(uuid).startswith("GPU-") else uuid
+    with ClockSampler(device.index if device.index is not None else 0, uuid=uuid) as clocks:
         for _ in range(args.warmup):
             step.run()
         torch.cuda.synchronize()
@@ -427,7 +556,12 @@ def run_ours(args):
         d2h = sum(o.numel() * o.element_size() for o in outs)
         e2e = {"value": whole_job_rate(step.gemm_flops / 1e12, world, e2e_ms / 1e3),
                "unit": "TFLOP/s", "h2d_bytes_per_step": step.h2d_bytes(),
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps}
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": e2e_steps,
+               "method": f"{e2e_steps} steps timed with CUDA events; each step copies X, W and "
+                         "dY of both linears from pinned host memory, queues the step's library "
+                         "calls through the C ABI (the three one-pass quantizations and three "
+                         "GEMMs per linear that the nvfp4_linear_* entry points make) and copies "
+                         "Y, dX and dW back to pinned host memory"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
