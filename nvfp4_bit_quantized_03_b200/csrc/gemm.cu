@@ -4,31 +4,35 @@
 // tecnico section 2, "Formato NVFP4": E2M1 operands with one E4M3 scale per 16 elements and
 // an FP32 scale per tensor, multiplied natively by Blackwell tensor cores.
 //
-// Design (one CTA per SM, persistent over 128 x 256 output tiles, 22 warps):
-//   warp 0      TMA producer: per 256-wide K block, the A (128 x 128 B) and B (256 x 128 B)
-//               code tiles with 128-byte swizzle, plus the block scales (contiguous 512-byte
-//               tiles of the MMA scale layout) by bulk copies, into a shared-memory ring of 4
-//               stages guarded by mbarriers.  The four MMAs of a stage take ~0.54 k cycles on
-//               the tensor pipe, while a stage's round trip (TMA ~1.7 k, scale staging
-//               ~0.55 k, issue ~0.5 k, MMAs + release ~1.1 k, more under load) spans several
-//               stages' MMA work: the kernel is bound by this operand feed, not by the MMAs.
-//   warps 2-5   scale stagers, one per 32-lane quarter of tensor memory: move each stage's
-//               scales shared -> registers -> tensor memory (ld.shared + tcgen05.st, into a
-//               per-stage column range), so the tensor pipe never spends time on scale copies.
-//   warp 1      TMEM owner and MMA issuer (one thread): tcgen05.mma kind::mxf4nvf4 (M 128,
-//               N 256, K 64, FP32 accumulation in TMEM; E4M3 scales, or UE8M0 for MXFP4
-//               operands), then commits the stage back to the producer.
-//   warps 6-21  epilogue: each warp drains one 32-lane quarter x 64 columns of the
-//               accumulator into registers (tcgen05.ld), releases the accumulator so the
-//               next tile's MMAs start at once, then scales by 1 / (S_enc,A S_enc,B) and
-//               writes the tile while the next one computes: bf16 rows through a 512-byte
-//               per-warp staging buffer with paced TMA bulk tensor stores (clipped at the
-//               matrix edge), FP32 pairs straight from registers with 8-byte stores.  With
-//               the fused amax, the bf16 epilogue also reduces max |D| and, by 16-lane
-//               shuffles across rows, max |RHT(D)| for the next quantization of D.
+// Design: persistent CTA pairs (clusters of two CTAs on one TPC), one per two SMs, over
+// 256 x 256 output tiles; each pair tile is one tcgen05.mma.cta_group::2 accumulation (M 256,
+// N 256, K 64 per instruction) whose A rows and B rows are split between the two CTAs, so each
+// SM reads 128 A rows and 128 B rows per K block: 38 KB per 256-wide K block where a single-CTA
+// 128 x 256 tile needs 54 KB for the same work.  22 warps per CTA:
+//   warp 0      TMA producer (both CTAs): per 256-wide K block, this CTA's A (128 x 128 B) and
+//               B (128 x 128 B) code boxes with 128-byte swizzle, this CTA's 128 rows of A
+//               scales and all 256 rows of B scales (contiguous 512-byte tiles of the MMA scale
+//               layout, bulk copies), into a shared-memory ring of 5 stages.
+//   warps 2-5   scale stagers, one per 32-lane quarter of tensor memory (both CTAs): move each
+//               stage's scales shared -> registers -> tensor memory (tcgen05.st), then arrive on
+//               the leader CTA's stage barrier.  (tcgen05.cp from the MMA thread would use the
+//               tensor pipe: measured on B200, twelve 32x128b copies per K block lengthen the
+//               block's four MMAs from 278 ns to 458 ns.)
+//   warp 1      tensor-memory owner (both CTAs, allocated for the pair) and, in the leader CTA,
+//               the MMA issuer (one thread): once both CTAs' stagers have arrived, four
+//               kind::mxf4nvf4 block-scaled MMAs (E4M3 scales, or UE8M0 for MXFP4 operands),
+//               then one commit that releases the stage in both CTAs.
+//   warps 6-21  epilogue (both CTAs): each warp drains one 32-lane quarter x 64 columns of its
+//               CTA's 128 x 256 half of the accumulator (tcgen05.ld), releases it to the leader,
+//               scales by 1 / (S_enc,A S_enc,B) and writes it while the next tile computes: bf16
+//               rows through a 512-byte per-warp staging buffer with paced TMA bulk tensor
+//               stores (clipped at the matrix edge), FP32 pairs straight from registers.  With
+//               the fused amax, the bf16 epilogue also reduces max |D| and, by 16-lane shuffles
+//               across rows, max |RHT(D)| for the next quantization of D.
+// No load is multicast: every CTA loads its own operands from this GPU's memory.
 // Every wait on an mbarrier is bounded in time; on expiry the kernel records
-// NVFP4_DEVSTAT_TIMEOUT, drains its in-flight copies and MMAs (again with a limit), frees
-// its tensor memory and returns.
+// NVFP4_DEVSTAT_TIMEOUT, drains its in-flight copies and MMAs (again with a limit), meets its
+// peer at a cluster barrier, frees its tensor memory and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -43,16 +47,18 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int BM = 128;                 // tile rows (A rows, TMEM lanes)
-constexpr int BN = 256;                 // tile columns (B rows, accumulator columns)
+constexpr int CTA_M = 128;              // A rows per CTA (tensor-memory lanes)
+constexpr int PAIR_M = 2 * CTA_M;       // rows of a pair tile
+constexpr int BN = 256;                 // columns of a pair tile (B rows), N of the MMA
+constexpr int B_ROWS = BN / 2;          // B rows each CTA loads
 constexpr int BK = 256;                 // K elements per pipeline stage (128 bytes per row)
 constexpr int MMA_K = 64;               // K per tcgen05.mma of kind::mxf4nvf4
-constexpr int A_BYTES = BM * BK / 2;    // 16 KB
-constexpr int B_BYTES = BN * BK / 2;    // 32 KB
+constexpr int A_BYTES = CTA_M * BK / 2;  // 16 KB
+constexpr int B_BYTES = B_ROWS * BK / 2;  // 16 KB
 constexpr int SF_TILE = 512;            // 128 rows x 4 blocks of scales
-constexpr int SFA_BYTES = (BM / 128) * (BK / MMA_K) * SF_TILE;  // 2 KB
-constexpr int SFB_BYTES = (BN / 128) * (BK / MMA_K) * SF_TILE;  // 4 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+constexpr int SFA_BYTES = (BK / MMA_K) * SF_TILE;      // 2 KB: this CTA's 128 A rows
+constexpr int SFB_BYTES = 2 * (BK / MMA_K) * SF_TILE;  // 4 KB: all 256 B rows of the tile
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 38 KB
 constexpr int NUM_SF_WARPS = 4;         // one per 32-lane quarter of tensor memory
 constexpr int NUM_EPI_WARPS = 16;       // four per lane quarter, 64 accumulator columns each
 constexpr int FIRST_SF_WARP = 2;
@@ -64,24 +70,24 @@ constexpr int SF_COL = BN;              // scales: 48 columns per stage from col
 constexpr int SF_COLS_PER_STAGE = (BK / MMA_K) * (4 + 8);
 constexpr int BAR_BYTES = 256;
 
-// Pipeline shape per output type.  Four operand stages either way: a bf16 tile (64 KB of
-// output) goes out through 512-byte staging buffers with paced TMA stores (a first-round delay
-// and a gap between rounds, so that they do not crowd the next tile's first operand loads); an
-// FP32 tile (128 KB) is stored straight from registers (store_f32_direct).
+// Pipeline shape per output type.  Five operand stages either way: a bf16 tile (64 KB of
+// output per CTA) goes out through 512-byte staging buffers with paced TMA stores (a
+// first-round delay and a gap between rounds, so that they do not crowd the next tile's first
+// operand loads); an FP32 tile (128 KB per CTA) is stored straight from registers.
 template <bool BF16>
 struct Pipe {
-    static constexpr int STAGES = 4;
+    static constexpr int STAGES = 5;
     static constexpr int STAGING_BYTES = 512;  // per epilogue warp (bf16 boxes; FP32 stores direct)
     static constexpr int SMEM_BYTES =
         STAGES * STAGE_BYTES + NUM_EPI_WARPS * STAGING_BYTES + BAR_BYTES + 1024;
     static constexpr unsigned FIRST_NS = BF16 ? 3000u : 0u;
     static constexpr unsigned GAP_NS = BF16 ? 1000u : 2000u;
-    // shared-memory barrier slots
-    static constexpr int BAR_FULL = 0;                     // [STAGES] TMA bytes of a stage landed
+    // shared-memory barrier slots (the same offsets in both CTAs of a pair)
+    static constexpr int BAR_FULL = 0;                     // [STAGES] this CTA's TMA bytes landed
     static constexpr int BAR_EMPTY = BAR_FULL + STAGES;    // [STAGES] the stage's MMAs completed
-    static constexpr int BAR_SF = BAR_EMPTY + STAGES;      // [STAGES] the stage's scales are in TMEM
+    static constexpr int BAR_SF = BAR_EMPTY + STAGES;      // [STAGES] leader: both CTAs' scales in TMEM
     static constexpr int BAR_ACC_FULL = BAR_SF + STAGES;   // the tile's accumulator is complete
-    static constexpr int BAR_ACC_EMPTY = BAR_ACC_FULL + 1; // the epilogue drained the accumulator
+    static constexpr int BAR_ACC_EMPTY = BAR_ACC_FULL + 1; // leader: both epilogues drained it
     static constexpr int BAR_DRAIN = BAR_ACC_EMPTY + 1;    // teardown after an abort
     static constexpr int NUM_BARS = BAR_DRAIN + 1;
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
@@ -94,10 +100,11 @@ constexpr int kDevTimeoutBit = 2;       // NVFP4_DEVSTAT_TIMEOUT
 static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment (128B swizzle)");
 
 // Instruction descriptor of tcgen05.mma kind::mxf4nvf4: A and B E2M1 (format 1), both
-// K-major, N >> 3 at bit 17, M >> 4 at bit 24, dense K = 64; bit 23 selects the scale type:
-// 0 = UE4M3 (NVFP4), 1 = UE8M0 (MXFP4, whose 32-block scales fill both 16-element slots).
+// K-major, N >> 3 at bit 17, M >> 4 at bit 24 (M = 256: the pair's rows), dense K = 64; bit 23
+// selects the scale type: 0 = UE4M3 (NVFP4), 1 = UE8M0 (MXFP4, whose 32-block scales fill both
+// 16-element slots).
 constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
-                           (static_cast<uint32_t>(BM >> 4) << 24);
+                           (static_cast<uint32_t>(PAIR_M >> 4) << 24);
 constexpr uint32_t IDESC_UE8M0 = IDESC | (1u << 23);
 
 struct Params {
@@ -136,9 +143,19 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
+// Arrive on the barrier at the same shared-memory offset in CTA `cta` of the cluster (this
+// CTA's own when cta is its rank).  The arrive keeps the default (CTA-scope release)
+// semantics: what it publishes to the peer is tensor-memory traffic, which the tcgen05 fences
+// around it order (tcgen05.fence::before_thread_sync here, ::after_thread_sync after the wait);
+// a cluster-scope release costs about half a microsecond per arrive on B200.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t cta)
 {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+    asm volatile(
+        "{\n\t.reg .b32 remote;\n\t"
+        "mapa.shared::cluster.u32 remote, %0, %1;\n\t"
+        "mbarrier.arrive.shared::cluster.b64 _, [remote];\n\t}" ::"r"(bar),
+        "r"(cta)
+        : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
@@ -152,14 +169,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
         : "memory");
     return ok != 0;
 }
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// All threads of both CTAs of the pair.
+__device__ __forceinline__ void cluster_sync()
+{
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 // Wait for the phase of `bar` with the given parity to complete.  Gives up when another
 // role has aborted (unless `ignore_abort`) or after WAIT_LIMIT_NS, which it reports.
-__device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* dev_status, bool ignore_abort = false,
-                                          unsigned long long limit_ns = WAIT_LIMIT_NS)
+__device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity,
+                                               volatile int* abort_flag, int* dev_status,
+                                               bool ignore_abort, unsigned long long limit_ns)
 {
-    if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
@@ -172,6 +200,15 @@ __device__ __noinline__ bool wait_bounded(uint32_t bar, uint32_t parity, volatil
             }
         }
     }
+}
+// The common case -- the phase has already completed -- costs one try_wait, inline.
+__device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
+                                             volatile int* abort_flag, int* dev_status,
+                                             bool ignore_abort = false,
+                                             unsigned long long limit_ns = WAIT_LIMIT_NS)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    return wait_bounded_slow(bar, parity, abort_flag, dev_status, ignore_abort, limit_ns);
 }
 
 // ---- TMA / bulk copies -------------------------------------------------------------------
@@ -247,24 +284,32 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* v)
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// One block-scaled MMA of the pair, issued by the leader CTA: D (256 x 256, rows 0-127 in the
+// leader's tensor memory, 128-255 in the peer's) += A . B^T over K = 64, where the descriptors'
+// shared-memory offsets select each CTA's 128 A rows and 128 B rows, and the scale addresses
+// each CTA's own scale columns (its A rows, all 256 B rows).
 template <bool MX>
-__device__ __forceinline__ void mma_nvf4(uint32_t d, uint64_t adesc, uint64_t bdesc,
-                                         uint32_t sfa, uint32_t sfb, uint32_t accumulate)
+__device__ __forceinline__ void mma_nvf4_pair(uint32_t d, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t sfa, uint32_t sfb, uint32_t accumulate)
 {
     constexpr uint32_t idesc = MX ? IDESC_UE8M0 : IDESC;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X "
+        "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.scale_vec::4X "
         "[%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
         : "memory");
 }
 
-__device__ __forceinline__ void mma_commit(uint32_t bar)
+// Arrive on the barrier at offset `bar` of both CTAs once every MMA the leader issued so far
+// has completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar)
 {
     asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+        "[%0], %1;" ::"r"(bar),
+        "h"(static_cast<uint16_t>(0x3))
         : "memory");
 }
 
@@ -355,11 +400,11 @@ __device__ __forceinline__ float apply_alpha(uint32_t acc_bits, const Alpha& al)
     return __fmul_rn(__fmul_rn(__uint_as_float(acc_bits), al.a1), al.a2);
 }
 
-// Output tile order: groups of 16 row tiles, column tiles inner, so that the CTAs working
-// at the same time share A and B tiles in L2.
+// Pair-tile order: groups of 8 row tiles (2048 rows), column tiles inner, so that the pairs
+// working at the same time share A and B tiles in L2.
 __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int& tm, int& tn)
 {
-    constexpr int G = 16;
+    constexpr int G = 8;
     const int group = t / (G * tiles_n);
     const int first = group * G;
     const int gsz = min(G, tiles_m - first);
@@ -478,7 +523,7 @@ __device__ __forceinline__ void store_f32_direct(const uint32_t* v, const Alpha&
 }
 
 template <bool BF16, bool MX, bool AMAX = false>
-__global__ void __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_d, const Params p)
@@ -489,6 +534,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr int BAR_ACC_FULL = P::BAR_ACC_FULL, BAR_ACC_EMPTY = P::BAR_ACC_EMPTY;
     constexpr int BAR_DRAIN = P::BAR_DRAIN, NUM_BARS = P::NUM_BARS;
     extern __shared__ uint8_t smem_raw[];
+    // Both CTAs of a pair lay out their shared memory identically: the MMA, the commits and
+    // the remote arrivals address the peer's buffers and barriers by the same offsets.
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     uint8_t* staging = smem + STAGES * STAGE_BYTES;
@@ -498,21 +545,24 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_m = (p.M + BM - 1) / BM, tiles_n = (p.N + BN - 1) / BN;
+    const uint32_t rank = cluster_rank();             // 0: leader (issues the MMAs), 1: peer
+    const int cluster = blockIdx.x >> 1, clusters = gridDim.x >> 1;
+    const int tiles_m = (p.M + PAIR_M - 1) / PAIR_M, tiles_n = (p.N + BN - 1) / BN;
     const int total = tiles_m * tiles_n;
     const int num_kb = (p.K + BK - 1) / BK;
     const int k_steps_total = p.K / MMA_K;
-    const int sf_groups = p.K / MMA_K;       // 4-block scale groups per row
+    const int sf_groups = p.K / MMA_K;                // 4-block scale groups per row
+    const int sfa_row_tiles = (p.M + 127) / 128;      // 128-row groups in A's scale buffer
     const int sfb_row_tiles = (p.N + 127) / 128;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(bar(BAR_FULL + s), 1);
             mbar_init(bar(BAR_EMPTY + s), 1);
-            mbar_init(bar(BAR_SF + s), NUM_SF_WARPS);
+            mbar_init(bar(BAR_SF + s), 2 * NUM_SF_WARPS);
         }
         mbar_init(bar(BAR_ACC_FULL), 1);
-        mbar_init(bar(BAR_ACC_EMPTY), NUM_EPI_WARPS);
+        mbar_init(bar(BAR_ACC_EMPTY), 2 * NUM_EPI_WARPS);
         mbar_init(bar(BAR_DRAIN), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -521,47 +571,56 @@ __global__ void __launch_bounds__(THREADS, 1)
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_d)) : "memory");
     }
     if (warp == 1) {
+        // one warp of each CTA allocates the pair's tensor memory (the same columns in both)
         __syncwarp();
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(tmem_slot)),
                      "r"(TMEM_COLS)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync();  // both CTAs' barriers are initialised before either signals the other
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0 && lane == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer (both CTAs) ----------------
         int stage = 0;
         uint32_t phase = 0;
         uint32_t issued[STAGES] = {};
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = cluster; t < total && ok; t += clusters) {
             int tm, tn;
             tile_coords(t, tiles_m, tiles_n, tm, tn);
+            const int ga = tm * 2 + static_cast<int>(rank);  // this CTA's 128-row group of A
+            const bool a_ok = ga < sfa_row_tiles;
+            const bool b_ok[2] = {2 * tn < sfb_row_tiles, 2 * tn + 1 < sfb_row_tiles};
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!wait_bounded(bar(BAR_EMPTY + stage), phase ^ 1, abort_flag, p.dev_status)) {
                     ok = false;
                     break;
                 }
                 const int natoms = min(BK / MMA_K, sf_groups - kb * (BK / MMA_K));
-                const bool b2 = (2 * tn + 1) < sfb_row_tiles;
-                const uint32_t sf_bytes = natoms * SF_TILE * (b2 ? 3u : 2u);
+                const uint32_t sf_bytes =
+                    natoms * SF_TILE * ((a_ok ? 1u : 0u) + (b_ok[0] ? 1u : 0u) + (b_ok[1] ? 1u : 0u));
                 const uint32_t full = bar(BAR_FULL + stage);
                 uint8_t* st = smem + stage * STAGE_BYTES;
                 mbar_expect_tx(full, A_BYTES + B_BYTES + sf_bytes);
-                tma_load_2d(smem_u32(st), &tmap_a, kb * (BK / 2), tm * BM, full);
-                tma_load_2d(smem_u32(st + A_BYTES), &tmap_b, kb * (BK / 2), tn * BN, full);
-                const size_t ga = (static_cast<size_t>(tm) * sf_groups + kb * (BK / MMA_K)) * SF_TILE;
-                bulk_load(smem_u32(st + A_BYTES + B_BYTES), p.sfa + ga, natoms * SF_TILE, full);
-                for (int h = 0; h < (b2 ? 2 : 1); ++h) {
-                    const size_t gb =
+                // boxes wholly or partly beyond M or N are zero-filled by the tensor maps
+                tma_load_2d(smem_u32(st), &tmap_a, kb * (BK / 2), ga * CTA_M, full);
+                tma_load_2d(smem_u32(st + A_BYTES), &tmap_b, kb * (BK / 2),
+                            tn * BN + static_cast<int>(rank) * B_ROWS, full);
+                if (a_ok) {
+                    const size_t off = (static_cast<size_t>(ga) * sf_groups + kb * (BK / MMA_K)) * SF_TILE;
+                    bulk_load(smem_u32(st + A_BYTES + B_BYTES), p.sfa + off, natoms * SF_TILE, full);
+                }
+                for (int h = 0; h < 2; ++h) {
+                    if (!b_ok[h]) continue;
+                    const size_t off =
                         (static_cast<size_t>(2 * tn + h) * sf_groups + kb * (BK / MMA_K)) * SF_TILE;
                     bulk_load(smem_u32(st + A_BYTES + B_BYTES + SFA_BYTES + h * (SFB_BYTES / 2)),
-                              p.sfb + gb, natoms * SF_TILE, full);
+                              p.sfb + off, natoms * SF_TILE, full);
                 }
                 ++issued[stage];
                 if (++stage == STAGES) {
@@ -576,20 +635,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (issued[s])
                     wait_bounded(bar(BAR_FULL + s), (issued[s] - 1) & 1, abort_flag, nullptr, true);
         }
-    } else if (warp == 1 && lane == 0) {
-        // ---------------- MMA issuer ----------------
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+        // ---------------- MMA issuer (leader CTA) ----------------
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true, any = false;
         int it = 0;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++it) {
+        for (int t = cluster; t < total && ok; t += clusters, ++it) {
+            // both CTAs' epilogues have drained the previous tile's accumulator
             if (!wait_bounded(bar(BAR_ACC_EMPTY), (it & 1) ^ 1, abort_flag, p.dev_status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
             for (int kb = 0; kb < num_kb; ++kb) {
-                // the stage's codes are in shared memory and its scales in tensor memory
+                // both CTAs' codes are in shared memory and their scales in tensor memory
                 if (!wait_bounded(bar(BAR_SF + stage), phase, abort_flag, p.dev_status)) {
                     ok = false;
                     break;
@@ -602,33 +662,40 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int k = 0; k < nk; ++k) {
                     // K step k = 64 elements = 32 bytes into the 128-byte swizzled rows; its
                     // scales: A in columns tcol + 4k, B in tcol + 16 + 8k
-                    mma_nvf4<MX>(tmem_base + ACC_COL, desc_sw128(a0 + 32 * k), desc_sw128(b0 + 32 * k),
-                             tcol + 4 * k, tcol + 16 + 8 * k, (kb | k) != 0 ? 1u : 0u);
+                    mma_nvf4_pair<MX>(tmem_base + ACC_COL, desc_sw128(a0 + 32 * k),
+                                      desc_sw128(b0 + 32 * k), tcol + 4 * k, tcol + 16 + 8 * k,
+                                      (kb | k) != 0 ? 1u : 0u);
                 }
                 any = true;
-                mma_commit(bar(BAR_EMPTY + stage));
+                mma_commit_pair(bar(BAR_EMPTY + stage));
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
                 }
             }
-            if (ok) mma_commit(bar(BAR_ACC_FULL));
+            if (ok) mma_commit_pair(bar(BAR_ACC_FULL));
         }
         if (!ok && any) {
-            mma_commit(bar(BAR_DRAIN));
+            mma_commit_pair(bar(BAR_DRAIN));
             wait_bounded(bar(BAR_DRAIN), 0, abort_flag, nullptr, true);
         }
     } else if (warp >= FIRST_SF_WARP && warp < FIRST_SF_WARP + NUM_SF_WARPS) {
-        // ---------------- scale stagers ----------------
-        // Tensor-memory layout the block-scaled MMA reads: row r's four E4M3 scales of one
-        // K step sit in lane r % 32 of every lane quarter, column r / 32.  Byte 16 l of a
-        // 512-byte scale tile holds exactly those 4 columns for rows l, l + 32, l + 64,
+        // ---------------- scale stagers (both CTAs) ----------------
+        // Tensor-memory layout the block-scaled MMA reads, in each CTA: row r's four E4M3
+        // scales of one K step sit in lane r % 32 of every lane quarter, column r / 32.  Byte
+        // 16 l of a 512-byte scale tile holds exactly those 4 columns for rows l, l + 32, l + 64,
         // l + 96, so lane l of each quarter's warp loads 16 bytes per tile and stores them.
+        // Scale tiles the producer did not load (row groups beyond M or N) are written as
+        // zeros, so the rows the TMA zero-filled multiply to zero, never to NaN.
         const int q = warp & 3;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int t = cluster; t < total && ok; t += clusters) {
+            int tm, tn;
+            tile_coords(t, tiles_m, tiles_n, tm, tn);
+            const bool a_ok = tm * 2 + static_cast<int>(rank) < sfa_row_tiles;
+            const bool b_ok[2] = {2 * tn < sfb_row_tiles, 2 * tn + 1 < sfb_row_tiles};
             for (int kb = 0; kb < num_kb; ++kb) {
                 bool ready = lane == 0 ? wait_bounded(bar(BAR_FULL + stage), phase, abort_flag,
                                                       p.dev_status)
@@ -643,7 +710,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint32_t ra[16], rb[32];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const uint4 v = *reinterpret_cast<const uint4*>(sf + k * SF_TILE + 16 * lane);
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (a_ok) v = *reinterpret_cast<const uint4*>(sf + k * SF_TILE + 16 * lane);
                     ra[4 * k] = v.x;
                     ra[4 * k + 1] = v.y;
                     ra[4 * k + 2] = v.z;
@@ -653,8 +721,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int k = 0; k < 4; ++k) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        const uint4 v = *reinterpret_cast<const uint4*>(
-                            sf + SFA_BYTES + h * (SFB_BYTES / 2) + k * SF_TILE + 16 * lane);
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (b_ok[h])
+                            v = *reinterpret_cast<const uint4*>(
+                                sf + SFA_BYTES + h * (SFB_BYTES / 2) + k * SF_TILE + 16 * lane);
                         const int c = 4 * (2 * k + h);
                         rb[c] = v.x;
                         rb[c + 1] = v.y;
@@ -669,7 +739,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tmem_wait_st();
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar(BAR_SF + stage));
+                if (lane == 0) mbar_arrive_cluster(bar(BAR_SF + stage), 0);
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
@@ -677,7 +747,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else if (warp >= FIRST_EPI_WARP) {
-        // ---------------- epilogue ----------------
+        // ---------------- epilogue (both CTAs) ----------------
         const int q = warp & 3;                         // TMEM lane quarter this warp may access
         const int chunk = (warp - FIRST_EPI_WARP) >> 2; // accumulator columns [64 chunk, +64)
         const uint32_t stage_buf = smem_u32(staging + (warp - FIRST_EPI_WARP) * STAGING_BYTES);
@@ -686,7 +756,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         int it = 0;
         uint32_t m_plain = 0, m_rht = 0;  // fused maxima (AMAX)
         const uint32_t flip = ((p.sign_mask >> (lane & 15)) & 1u) ? 0x80000000u : 0u;
-        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+        for (int t = cluster; t < total; t += clusters, ++it) {
             // one lane waits, so the whole warp takes the same branch into tcgen05.ld
             bool ready = lane == 0 ? wait_bounded(bar(BAR_ACC_FULL), it & 1, abort_flag,
                                                   p.dev_status)
@@ -710,11 +780,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar(BAR_ACC_EMPTY));
+            if (lane == 0) mbar_arrive_cluster(bar(BAR_ACC_EMPTY), 0);
 
             int tm, tn;
             tile_coords(t, tiles_m, tiles_n, tm, tn);
-            const int y = tm * BM + 32 * q;       // first output row of this warp's slice
+            // first output row of this warp's slice: the CTA's half of the pair tile
+            const int y = tm * PAIR_M + static_cast<int>(rank) * CTA_M + 32 * q;
             const int n0 = tn * BN + 64 * chunk;  // first output column
             if (BF16)
                 store_slice<BF16, AMAX>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N,
@@ -734,12 +805,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
 
+    // Neither CTA frees its tensor memory or exits while the pair's MMAs or the peer's
+    // arrivals may still reach it.
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     if (warp == 1) {
         __syncwarp();
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(TMEM_COLS)
                      : "memory");
     }
@@ -777,7 +851,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
 }
 
 // 2D map over a codes buffer (rows x K/2 bytes), boxes of `box_rows` x 128 bytes, 128-byte
-// swizzle, zero fill outside the tensor.
+// swizzle, zero fill outside the tensor (boxes may start beyond the last row).
 bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_t K, int box_rows)
 {
     auto enc = tensor_map_encoder();
@@ -819,32 +893,49 @@ cudaError_t launch_wait_selftest(int* dev_status, unsigned long long limit_ns, c
 
 cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
 {
-    // the kernels' shared-memory limit is raised once per device
+    // Once per device: the kernels' shared-memory limit is raised and the number of CTA pairs
+    // that can be resident at once is looked up (the persistent grid is one wave of pairs).
     constexpr int kDevices = 64;
-    static bool configured[kDevices] = {};
+    static int max_pairs[kDevices] = {};
     static std::mutex configure_mutex;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices)
         return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(configure_mutex);
-    if (!configured[dev]) {
-        cudaError_t e = cudaSuccess;
-        const void* kernels[5] = {reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false>),
-                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<false, false>),
-                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<true, true>),
-                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<false, true>),
-                                  reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false, true>)};
-        const int smem[5] = {Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
-                             Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
-                             Pipe<true>::SMEM_BYTES};
-        for (int i = 0; i < 5 && e == cudaSuccess; ++i)
-            e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     smem[i]);
-        if (e != cudaSuccess) return e;
-        configured[dev] = true;
+    {
+        std::lock_guard<std::mutex> lock(configure_mutex);
+        if (max_pairs[dev] == 0) {
+            cudaError_t e = cudaSuccess;
+            const void* kernels[5] = {
+                reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false>),
+                reinterpret_cast<const void*>(gemm_nvf4_kernel<false, false>),
+                reinterpret_cast<const void*>(gemm_nvf4_kernel<true, true>),
+                reinterpret_cast<const void*>(gemm_nvf4_kernel<false, true>),
+                reinterpret_cast<const void*>(gemm_nvf4_kernel<true, false, true>)};
+            const int smem[5] = {Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
+                                 Pipe<true>::SMEM_BYTES, Pipe<false>::SMEM_BYTES,
+                                 Pipe<true>::SMEM_BYTES};
+            for (int i = 0; i < 5 && e == cudaSuccess; ++i)
+                e = cudaFuncSetAttribute(kernels[i], cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem[i]);
+            if (e != cudaSuccess) return e;
+            int pairs = 0;
+            for (int i = 0; i < 5; ++i) {
+                cudaLaunchConfig_t cfg = {};
+                cfg.gridDim = dim3(static_cast<unsigned>(sm_count & ~1), 1, 1);
+                cfg.blockDim = dim3(THREADS, 1, 1);
+                cfg.dynamicSmemBytes = static_cast<size_t>(smem[i]);
+                int n = 0;
+                if (cudaOccupancyMaxActiveClusters(&n, kernels[i], &cfg) != cudaSuccess || n < 1)
+                    n = sm_count / 2;
+                pairs = (i == 0 || n < pairs) ? n : pairs;
+            }
+            (void)cudaGetLastError();  // a failed occupancy query leaves no sticky error
+            max_pairs[dev] = pairs > 0 ? pairs : 1;
+        }
     }
     CUtensorMap ma, mb, md;
-    if (!make_codes_map(&ma, g.a_codes, g.M, g.K, BM) || !make_codes_map(&mb, g.b_codes, g.N, g.K, BN) ||
+    if (!make_codes_map(&ma, g.a_codes, g.M, g.K, CTA_M) ||
+        !make_codes_map(&mb, g.b_codes, g.N, g.K, B_ROWS) ||
         !make_output_map(&md, g.D, g.M, g.N, g.ldd, g.out_bf16 != 0))
         return cudaErrorInvalidValue;
     Params p;
@@ -861,8 +952,9 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
     p.dev_status = g.dev_status;
     p.amax_out = g.amax_out;
     p.sign_mask = g.sign_mask;
-    const int64_t tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
-    const int grid = static_cast<int>(tiles < sm_count ? tiles : sm_count);
+    const int64_t tiles = ((g.M + PAIR_M - 1) / PAIR_M) * ((g.N + BN - 1) / BN);
+    const int pairs = static_cast<int>(tiles < max_pairs[dev] ? tiles : max_pairs[dev]);
+    const int grid = 2 * pairs;  // clusters of two CTAs (__cluster_dims__)
     if (g.amax_out) {
         // fused maxima of the bf16 output for the next quantizer (the API allows it only there)
         if (!g.out_bf16 || g.mx) return cudaErrorInvalidValue;
