@@ -87,11 +87,11 @@ struct Pipe {
     static constexpr int BAR_EMPTY = BAR_FULL + STAGES;    // [STAGES] the stage's MMAs completed
     static constexpr int BAR_SF = BAR_EMPTY + STAGES;      // [STAGES] leader: both CTAs' scales in TMEM
     static constexpr int BAR_ACC_FULL = BAR_SF + STAGES;   // the tile's accumulator is complete
-    static constexpr int BAR_ACC_EMPTY = BAR_ACC_FULL + 1; // leader: both epilogues drained it
+    static constexpr int BAR_ACC_EMPTY = BAR_ACC_FULL + 1; // leader: both CTAs' epilogues drained it
     static constexpr int BAR_DRAIN = BAR_ACC_EMPTY + 1;    // teardown after an abort
     static constexpr int NUM_BARS = BAR_DRAIN + 1;
     static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
-    static_assert(NUM_BARS * 8 + 16 <= BAR_BYTES, "barrier area");
+    static_assert(NUM_BARS * 8 + 16 <= BAR_BYTES, "barrier area (+ TMEM slot, abort and go flags)");
     static_assert(SF_COL + STAGES * SF_COLS_PER_STAGE <= TMEM_COLS, "tensor memory budget");
 };
 constexpr unsigned long long WAIT_LIMIT_NS = 2000000000ull;  // 2 s per wait
@@ -110,8 +110,6 @@ constexpr uint32_t IDESC_UE8M0 = IDESC | (1u << 23);
 struct Params {
     uint32_t* amax_out;  // fused maxima (bf16 output only): [max |D|, max |RHT(D)|] as FP32 bits
     uint32_t sign_mask;  // RHT signs for amax_out[1]
-    const uint8_t* sfa;
-    const uint8_t* sfb;
     const float* amax_a;
     const float* amax_b;
     void* D;
@@ -157,6 +155,19 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t cta)
         "r"(cta)
         : "memory");
 }
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
 {
     uint32_t ok;
@@ -201,6 +212,33 @@ __device__ __noinline__ bool wait_bounded_slow(uint32_t bar, uint32_t parity,
         }
     }
 }
+// For the accumulator hand-off between the MMA issuer and the epilogue, where the waiting
+// thread is alone and the wake-up latency of a suspended try_wait shows in every tile: spin on
+// the non-blocking test, with the same time limit and abort handling as wait_bounded.
+__device__ __noinline__ bool wait_spin(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                       int* dev_status)
+{
+    if (mbar_test_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test_wait(bar, parity)) return true;
+        if ((i & 63u) == 0) {
+            if (*abort_flag) return false;
+            if (globaltimer() - t0 > WAIT_LIMIT_NS) {
+                *abort_flag = 1;
+                if (dev_status) atomicOr(dev_status, kDevTimeoutBit);
+                return false;
+            }
+        }
+    }
+}
+
+// Named barrier among `threads` threads (whole warps), id 1..15.
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t threads)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // The common case -- the phase has already completed -- costs one try_wait, inline.
 __device__ __forceinline__ bool wait_bounded(uint32_t bar, uint32_t parity,
                                              volatile int* abort_flag, int* dev_status,
@@ -221,13 +259,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
         : "memory");
 }
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar)
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x,
+                                            int32_t y, int32_t z, uint32_t bar)
 {
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
-            "r"(dst),
-        "l"(src), "r"(bytes), "r"(bar)
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+        "[%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
         : "memory");
 }
 
@@ -526,6 +564,8 @@ template <bool BF16, bool MX, bool AMAX = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     gemm_nvf4_kernel(const __grid_constant__ CUtensorMap tmap_a,
                      const __grid_constant__ CUtensorMap tmap_b,
+                     const __grid_constant__ CUtensorMap tmap_sfa,
+                     const __grid_constant__ CUtensorMap tmap_sfb,
                      const __grid_constant__ CUtensorMap tmap_d, const Params p)
 {
     using P = Pipe<BF16>;
@@ -542,6 +582,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     uint64_t* bars = reinterpret_cast<uint64_t*>(staging + NUM_EPI_WARPS * STAGING_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    volatile int* epi_go = abort_flag + 1;  // the epilogue's waiter tells the other warps
     auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -551,9 +592,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int total = tiles_m * tiles_n;
     const int num_kb = (p.K + BK - 1) / BK;
     const int k_steps_total = p.K / MMA_K;
-    const int sf_groups = p.K / MMA_K;                // 4-block scale groups per row
-    const int sfa_row_tiles = (p.M + 127) / 128;      // 128-row groups in A's scale buffer
-    const int sfb_row_tiles = (p.N + 127) / 128;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -562,12 +600,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_init(bar(BAR_SF + s), 2 * NUM_SF_WARPS);
         }
         mbar_init(bar(BAR_ACC_FULL), 1);
-        mbar_init(bar(BAR_ACC_EMPTY), 2 * NUM_EPI_WARPS);
+        mbar_init(bar(BAR_ACC_EMPTY), 2);  // one arrival per CTA's epilogue
         mbar_init(bar(BAR_DRAIN), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_sfa)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_sfb)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_d)) : "memory");
     }
     if (warp == 1) {
@@ -586,43 +626,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer (both CTAs) ----------------
+        // Four copies per stage: this CTA's A box and B box (128 rows x 128 bytes each, 128-byte
+        // swizzle) and two boxes of the scale maps: this CTA's 128 A rows and both 128-row
+        // groups of the tile's B rows, 4 scale tiles (one 256-wide K block) each.  Every box is
+        // full size: the maps zero-fill rows, row groups and K tiles beyond the matrices.
         int stage = 0;
         uint32_t phase = 0;
-        uint32_t issued[STAGES] = {};
+        uint32_t fills = 0;  // stages filled so far
         bool ok = true;
         for (int t = cluster; t < total && ok; t += clusters) {
             int tm, tn;
             tile_coords(t, tiles_m, tiles_n, tm, tn);
             const int ga = tm * 2 + static_cast<int>(rank);  // this CTA's 128-row group of A
-            const bool a_ok = ga < sfa_row_tiles;
-            const bool b_ok[2] = {2 * tn < sfb_row_tiles, 2 * tn + 1 < sfb_row_tiles};
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!wait_bounded(bar(BAR_EMPTY + stage), phase ^ 1, abort_flag, p.dev_status)) {
                     ok = false;
                     break;
                 }
-                const int natoms = min(BK / MMA_K, sf_groups - kb * (BK / MMA_K));
-                const uint32_t sf_bytes =
-                    natoms * SF_TILE * ((a_ok ? 1u : 0u) + (b_ok[0] ? 1u : 0u) + (b_ok[1] ? 1u : 0u));
                 const uint32_t full = bar(BAR_FULL + stage);
-                uint8_t* st = smem + stage * STAGE_BYTES;
-                mbar_expect_tx(full, A_BYTES + B_BYTES + sf_bytes);
-                // boxes wholly or partly beyond M or N are zero-filled by the tensor maps
-                tma_load_2d(smem_u32(st), &tmap_a, kb * (BK / 2), ga * CTA_M, full);
-                tma_load_2d(smem_u32(st + A_BYTES), &tmap_b, kb * (BK / 2),
+                const uint32_t st = smem_u32(smem + stage * STAGE_BYTES);
+                mbar_expect_tx(full, STAGE_BYTES);
+                tma_load_2d(st, &tmap_a, kb * (BK / 2), ga * CTA_M, full);
+                tma_load_2d(st + A_BYTES, &tmap_b, kb * (BK / 2),
                             tn * BN + static_cast<int>(rank) * B_ROWS, full);
-                if (a_ok) {
-                    const size_t off = (static_cast<size_t>(ga) * sf_groups + kb * (BK / MMA_K)) * SF_TILE;
-                    bulk_load(smem_u32(st + A_BYTES + B_BYTES), p.sfa + off, natoms * SF_TILE, full);
-                }
-                for (int h = 0; h < 2; ++h) {
-                    if (!b_ok[h]) continue;
-                    const size_t off =
-                        (static_cast<size_t>(2 * tn + h) * sf_groups + kb * (BK / MMA_K)) * SF_TILE;
-                    bulk_load(smem_u32(st + A_BYTES + B_BYTES + SFA_BYTES + h * (SFB_BYTES / 2)),
-                              p.sfb + off, natoms * SF_TILE, full);
-                }
-                ++issued[stage];
+                tma_load_3d(st + A_BYTES + B_BYTES, &tmap_sfa, 0, kb * (BK / MMA_K), ga, full);
+                tma_load_3d(st + A_BYTES + B_BYTES + SFA_BYTES, &tmap_sfb, 0, kb * (BK / MMA_K),
+                            2 * tn, full);
+                ++fills;
                 if (++stage == STAGES) {
                     stage = 0;
                     phase ^= 1;
@@ -630,50 +660,88 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
         }
         if (!ok) {
-            // Let every copy already issued land before the CTA can exit.
-            for (int s = 0; s < STAGES; ++s)
-                if (issued[s])
-                    wait_bounded(bar(BAR_FULL + s), (issued[s] - 1) & 1, abort_flag, nullptr, true);
+            // Let every copy already issued land before the CTA can exit: slot s was filled
+            // n_s times, and its last fill completes phase n_s - 1 of its full barrier.
+            for (int s = 0; s < STAGES; ++s) {
+                const uint32_t n_s = fills > static_cast<uint32_t>(s)
+                                         ? (fills - static_cast<uint32_t>(s) + STAGES - 1) / STAGES
+                                         : 0u;
+                if (n_s) wait_bounded(bar(BAR_FULL + s), (n_s - 1) & 1, abort_flag, nullptr, true);
+            }
         }
     } else if (warp == 1 && lane == 0 && rank == 0) {
         // ---------------- MMA issuer (leader CTA) ----------------
-        int stage = 0;
+        // The MMA instructions issue at about the rate the tensor pipe executes them, so every
+        // instruction this thread runs between two K blocks leaves the pipe idle.  The loop is
+        // unrolled over the ring's slots, which it visits in order across tiles as the producer
+        // and the stagers do, so each slot's descriptors, scale columns and barriers are
+        // constants; the next slot's barrier is tested (and the fence taken) before this slot's
+        // last MMA, and the commit follows it.  Descriptors address shared memory through a
+        // 14-bit start-address field (address / 16): a slot is STAGE_BYTES / 16 further on, a K
+        // step 32 bytes (2 units).
+        const uint32_t s0 = smem_u32(smem);
+        uint64_t da[STAGES], db[STAGES];
+        uint32_t tc[STAGES];
+#pragma unroll
+        for (int j = 0; j < STAGES; ++j) {
+            da[j] = desc_sw128(s0 + j * STAGE_BYTES);
+            db[j] = desc_sw128(s0 + j * STAGE_BYTES + A_BYTES);
+            tc[j] = tmem_base + SF_COL + j * SF_COLS_PER_STAGE;
+        }
+        const uint32_t acc = tmem_base + ACC_COL;
+        const bool k_full = (k_steps_total % (BK / MMA_K)) == 0;  // every stage has 4 K steps
         uint32_t phase = 0;
         bool ok = true, any = false;
-        int it = 0;
-        for (int t = cluster; t < total && ok; t += clusters, ++it) {
-            // both CTAs' epilogues have drained the previous tile's accumulator
-            if (!wait_bounded(bar(BAR_ACC_EMPTY), (it & 1) ^ 1, abort_flag, p.dev_status)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            for (int kb = 0; kb < num_kb; ++kb) {
-                // both CTAs' codes are in shared memory and their scales in tensor memory
-                if (!wait_bounded(bar(BAR_SF + stage), phase, abort_flag, p.dev_status)) {
-                    ok = false;
-                    break;
+        int it = 0, kb = 0, t = cluster;
+        bool live = t < total;
+        while (live && ok) {
+#pragma unroll
+            for (int j = 0; j < STAGES; ++j) {
+                if (!live || !ok) break;
+                if (kb == 0) {
+                    // tile start: both CTAs' epilogues have drained the previous accumulator,
+                    // and this slot's operands and scales are in place
+                    if (!wait_spin(bar(BAR_ACC_EMPTY), (it & 1) ^ 1, abort_flag, p.dev_status) ||
+                        !wait_bounded(bar(BAR_SF + j), phase, abort_flag, p.dev_status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
                 }
-                tc_fence_after();
-                const uint8_t* st = smem + stage * STAGE_BYTES;
-                const uint32_t a0 = smem_u32(st), b0 = smem_u32(st + A_BYTES);
-                const uint32_t tcol = tmem_base + SF_COL + stage * SF_COLS_PER_STAGE;
-                const int nk = min(BK / MMA_K, k_steps_total - kb * (BK / MMA_K));
-                for (int k = 0; k < nk; ++k) {
-                    // K step k = 64 elements = 32 bytes into the 128-byte swizzled rows; its
-                    // scales: A in columns tcol + 4k, B in tcol + 16 + 8k
-                    mma_nvf4_pair<MX>(tmem_base + ACC_COL, desc_sw128(a0 + 32 * k),
-                                      desc_sw128(b0 + 32 * k), tcol + 4 * k, tcol + 16 + 8 * k,
-                                      (kb | k) != 0 ? 1u : 0u);
+                const bool more = kb + 1 < num_kb;
+                const int jn = j + 1 == STAGES ? 0 : j + 1;
+                const uint32_t pn = j + 1 == STAGES ? phase ^ 1 : phase;
+                // K step k: scales of A in columns tc + 4k, of B in tc + 16 + 8k
+                if (k_full || more) {
+                    mma_nvf4_pair<MX>(acc, da[j], db[j], tc[j], tc[j] + 16, kb != 0 ? 1u : 0u);
+                    mma_nvf4_pair<MX>(acc, da[j] + 2, db[j] + 2, tc[j] + 4, tc[j] + 24, 1u);
+                    mma_nvf4_pair<MX>(acc, da[j] + 4, db[j] + 4, tc[j] + 8, tc[j] + 32, 1u);
+                    if (more) {
+                        if (!mbar_test_wait(bar(BAR_SF + jn), pn) &&
+                            !wait_bounded(bar(BAR_SF + jn), pn, abort_flag, p.dev_status))
+                            ok = false;
+                        tc_fence_after();
+                    }
+                    mma_nvf4_pair<MX>(acc, da[j] + 6, db[j] + 6, tc[j] + 12, tc[j] + 40, 1u);
+                } else {
+                    const int nk = k_steps_total - kb * (BK / MMA_K);  // 1..3 K steps left
+                    for (int k = 0; k < nk; ++k)
+                        mma_nvf4_pair<MX>(acc, da[j] + 2 * k, db[j] + 2 * k, tc[j] + 4 * k,
+                                          tc[j] + 16 + 8 * k, (kb | k) != 0 ? 1u : 0u);
                 }
                 any = true;
-                mma_commit_pair(bar(BAR_EMPTY + stage));
-                if (++stage == STAGES) {
-                    stage = 0;
-                    phase ^= 1;
+                mma_commit_pair(bar(BAR_EMPTY + j));
+                if (!more) {
+                    if (ok) mma_commit_pair(bar(BAR_ACC_FULL));
+                    kb = 0;
+                    ++it;
+                    t += clusters;
+                    live = t < total;
+                } else {
+                    ++kb;
                 }
             }
-            if (ok) mma_commit_pair(bar(BAR_ACC_FULL));
+            phase ^= 1;
         }
         if (!ok && any) {
             mma_commit_pair(bar(BAR_DRAIN));
@@ -685,17 +753,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // scales of one K step sit in lane r % 32 of every lane quarter, column r / 32.  Byte
         // 16 l of a 512-byte scale tile holds exactly those 4 columns for rows l, l + 32, l + 64,
         // l + 96, so lane l of each quarter's warp loads 16 bytes per tile and stores them.
-        // Scale tiles the producer did not load (row groups beyond M or N) are written as
-        // zeros, so the rows the TMA zero-filled multiply to zero, never to NaN.
+        // Row groups beyond M or N and K tiles beyond K arrive zero-filled from the scale maps,
+        // so padding rows (whose codes are zero-filled too) multiply to zero, never to NaN.
         const int q = warp & 3;
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
         for (int t = cluster; t < total && ok; t += clusters) {
-            int tm, tn;
-            tile_coords(t, tiles_m, tiles_n, tm, tn);
-            const bool a_ok = tm * 2 + static_cast<int>(rank) < sfa_row_tiles;
-            const bool b_ok[2] = {2 * tn < sfb_row_tiles, 2 * tn + 1 < sfb_row_tiles};
             for (int kb = 0; kb < num_kb; ++kb) {
                 bool ready = lane == 0 ? wait_bounded(bar(BAR_FULL + stage), phase, abort_flag,
                                                       p.dev_status)
@@ -710,8 +774,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 uint32_t ra[16], rb[32];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (a_ok) v = *reinterpret_cast<const uint4*>(sf + k * SF_TILE + 16 * lane);
+                    const uint4 v = *reinterpret_cast<const uint4*>(sf + k * SF_TILE + 16 * lane);
                     ra[4 * k] = v.x;
                     ra[4 * k + 1] = v.y;
                     ra[4 * k + 2] = v.z;
@@ -721,10 +784,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 for (int k = 0; k < 4; ++k) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (b_ok[h])
-                            v = *reinterpret_cast<const uint4*>(
-                                sf + SFA_BYTES + h * (SFB_BYTES / 2) + k * SF_TILE + 16 * lane);
+                        const uint4 v = *reinterpret_cast<const uint4*>(
+                            sf + SFA_BYTES + h * (SFB_BYTES / 2) + k * SF_TILE + 16 * lane);
                         const int c = 4 * (2 * k + h);
                         rb[c] = v.x;
                         rb[c + 1] = v.y;
@@ -756,14 +817,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         int it = 0;
         uint32_t m_plain = 0, m_rht = 0;  // fused maxima (AMAX)
         const uint32_t flip = ((p.sign_mask >> (lane & 15)) & 1u) ? 0x80000000u : 0u;
+        constexpr uint32_t EPI_THREADS = 32 * NUM_EPI_WARPS;
+        const bool waiter = warp == FIRST_EPI_WARP && lane == 0;
         for (int t = cluster; t < total; t += clusters, ++it) {
-            // one lane waits, so the whole warp takes the same branch into tcgen05.ld
-            bool ready = lane == 0 ? wait_bounded(bar(BAR_ACC_FULL), it & 1, abort_flag,
-                                                  p.dev_status)
-                                   : false;
-            ready = __shfl_sync(0xFFFFFFFFu, ready ? 1 : 0, 0) != 0;
-            if (!ready) break;
-            __syncwarp();
+            // one thread spins on the accumulator barrier and releases the other epilogue
+            // warps through a named barrier (a hardware barrier: nobody else polls)
+            if (waiter) *epi_go = wait_spin(bar(BAR_ACC_FULL), it & 1, abort_flag, p.dev_status);
+            named_sync(1, EPI_THREADS);
+            if (!*epi_go) break;
             tc_fence_after();
             uint32_t v[64];
             const uint32_t taddr = tmem_base + ACC_COL + (static_cast<uint32_t>(32 * q) << 16) +
@@ -779,8 +840,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             tmem_wait_ld();
             tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(bar(BAR_ACC_EMPTY), 0);
+            // every epilogue warp holds its slice: one arrival releases the accumulator
+            named_sync(2, EPI_THREADS);
+            if (waiter) mbar_arrive_cluster(bar(BAR_ACC_EMPTY), 0);
 
             int tm, tn;
             tile_coords(t, tiles_m, tiles_n, tm, tn);
@@ -865,6 +927,23 @@ bool make_codes_map(CUtensorMap* map, const uint8_t* codes, int64_t rows, int64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3D map over a scale buffer in the MMA layout, as 32-bit words: x = the 128 words of one
+// 512-byte tile, y = the K tile (4 blocks = 64 elements of K), z = the 128-row group; boxes of
+// 4 K tiles x `groups` row groups, zero fill beyond the buffer (ragged K, padding groups).
+bool make_scales_map(CUtensorMap* map, const uint8_t* scales, int64_t rows, int64_t K, int groups)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {SF_TILE / 4, static_cast<cuuint64_t>(K / MMA_K),
+                                static_cast<cuuint64_t>((rows + 127) / 128)};
+    const cuuint64_t strides[2] = {SF_TILE, static_cast<cuuint64_t>(K / MMA_K) * SF_TILE};
+    const cuuint32_t box[3] = {SF_TILE / 4, BK / MMA_K, static_cast<cuuint32_t>(groups)};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<uint8_t*>(scales), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2D map over D (rows x N elements, row stride ldd) for the epilogue's bulk tensor stores
 // (the map clips rows beyond M): bf16 boxes of 32 rows x 16 bytes, unswizzled; FP32 boxes of
 // 32 rows x 64 bytes with the 64-byte swizzle.
@@ -933,14 +1012,14 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
             max_pairs[dev] = pairs > 0 ? pairs : 1;
         }
     }
-    CUtensorMap ma, mb, md;
+    CUtensorMap ma, mb, msa, msb, md;
     if (!make_codes_map(&ma, g.a_codes, g.M, g.K, CTA_M) ||
         !make_codes_map(&mb, g.b_codes, g.N, g.K, B_ROWS) ||
+        !make_scales_map(&msa, g.a_scales, g.M, g.K, 1) ||
+        !make_scales_map(&msb, g.b_scales, g.N, g.K, 2) ||
         !make_output_map(&md, g.D, g.M, g.N, g.ldd, g.out_bf16 != 0))
         return cudaErrorInvalidValue;
     Params p;
-    p.sfa = g.a_scales;
-    p.sfb = g.b_scales;
     p.amax_a = g.a_amax;
     p.amax_b = g.b_amax;
     p.D = g.D;
@@ -961,15 +1040,15 @@ cudaError_t launch_gemm(const GemmArgs& g, int sm_count, cudaStream_t s)
         const cudaError_t e = cudaMemsetAsync(g.amax_out, 0, 2 * sizeof(uint32_t), s);
         if (e != cudaSuccess) return e;
         gemm_nvf4_kernel<true, false, true>
-            <<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
+            <<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, msa, msb, md, p);
     } else if (g.out_bf16 && !g.mx)
-        gemm_nvf4_kernel<true, false><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
+        gemm_nvf4_kernel<true, false><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, msa, msb, md, p);
     else if (!g.mx)
-        gemm_nvf4_kernel<false, false><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, md, p);
+        gemm_nvf4_kernel<false, false><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, msa, msb, md, p);
     else if (g.out_bf16)
-        gemm_nvf4_kernel<true, true><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, md, p);
+        gemm_nvf4_kernel<true, true><<<grid, THREADS, Pipe<true>::SMEM_BYTES, s>>>(ma, mb, msa, msb, md, p);
     else
-        gemm_nvf4_kernel<false, true><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, md, p);
+        gemm_nvf4_kernel<false, true><<<grid, THREADS, Pipe<false>::SMEM_BYTES, s>>>(ma, mb, msa, msb, md, p);
     return cudaGetLastError();
 }
 
