@@ -807,7 +807,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
         }
-    } else if (warp >= FIRST_EPI_WARP) {
+    } else if (warp >= FIRST_EPI_WARP && warp < FIRST_EPI_WARP + NUM_EPI_WARPS) {
         // ---------------- epilogue (both CTAs) ----------------
         const int q = warp & 3;                         // TMEM lane quarter this warp may access
         const int chunk = (warp - FIRST_EPI_WARP) >> 2; // accumulator columns [64 chunk, +64)
