@@ -202,16 +202,16 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi)
 // the lower neighbour.  Then i + [r16 < 65536 p] = ceil(mu(a) - r16 / 65536): for an integer
 // r16, r16 < 65536 p holds iff p - r16 / 65536 > 0.  The kernel evaluates it exactly on the
 // 65536-scaled values m = 65536 mu(a):
-//   * the lines a * 2^17 (exact), a * 2^16 + 2^17 and a * 2^15 + 2^18 rounded upward, and the
-//     constant 7 * 2^16: their minimum m' lies in [m, RU(m)];
-//   * P = RU(m' + 2^23) = 2^23 + ceil(m) (the spacing of FP32 at 2^23 is 1, and every
-//     integer from m up to ceil(m) is representable, so rounding m up first changes nothing);
+//   * the lines a * 2^17, a * 2^16 + 2^17 and a * 2^15 + 2^18, each plus 2^23 and rounded
+//     upward by one FMA, and the constant 2^23 + 7 * 2^16: below 2^24 the FP32 spacing is 1, so
+//     each rounded line is 2^23 + ceil(line), and since ceil is monotone their minimum is
+//     P = 2^23 + ceil(m) (for a >= 6 the constant is the minimum: code 7);
 //   * Q = P - (2^23 + r16) = ceil(m) - r16, exact (integers below 2^24);
-//   * k = RU(Q / 2^16 + 1.5 * 2^23) = 1.5 * 2^23 + ceil(Q / 2^16) = 1.5 * 2^23 + code
+//   * k = RU(Q / 2^16 + 1.5 * 2^23) = 1.5 * 2^23 + code
 //     (ceil(ceil(m) - r16) / 2^16) = ceil((m - r16) / 2^16) for integer r16, and Q / 2^16 lies
 //     in (-1, 7], where FP32 spacing is 1 around 1.5 * 2^23).
-// The low byte of k's bit pattern is the magnitude code.  Every operation is an FP32 FMA-pipe
-// instruction with a fixed rounding direction, so the result does not depend on contraction.
+// The pattern of k is 0x4B400000 + code.  Every operation is an FP32 FMA-pipe instruction
+// with a fixed rounding direction, so the result does not depend on contraction.
 
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel)
 {
@@ -238,21 +238,24 @@ __device__ __forceinline__ uint32_t rand16_as_f32_bits(uint32_t word, int h)
 // rbits = bits(2^23 + r16); the code is the low byte of the returned pattern.
 __device__ __forceinline__ uint32_t e2m1_sr_code(float a, uint32_t rbits)
 {
-    const float l0 = __fmul_rn(a, 131072.0f);
-    const float l1 = __fmaf_ru(a, 65536.0f, 131072.0f);
-    const float l2 = __fmaf_ru(a, 32768.0f, 262144.0f);
-    const float m = fminf(min3f(l0, l1, l2), 458752.0f);
-    const float P = __fadd_ru(m, 8388608.0f);
+    const float l0 = __fmaf_ru(a, 131072.0f, 8388608.0f);  // 2^23 + 2^17 a
+    const float l1 = __fmaf_ru(a, 65536.0f, 8519680.0f);   // 2^23 + 2^16 a + 2^17
+    const float l2 = __fmaf_ru(a, 32768.0f, 8650752.0f);   // 2^23 + 2^15 a + 2^18
+    const float P = fminf(min3f(l0, l1, l2), 8847360.0f);  // 2^23 + 7 * 2^16
     const float Q = __fsub_rn(P, __uint_as_float(rbits));
     return __float_as_uint(__fmaf_ru(Q, 0x1p-16f, 12582912.0f));
 }
 
-// Eight codes held in the low bytes of k[0..7] packed as nibbles, element j at bits 4j..4j+3.
+// Eight codes from the patterns k[j] = 0x4B400000 + code_j packed as nibbles, element j at
+// bits 4j..4j+3: sum_j k[j] 16^j, minus the sum of the constant parts, 0x4B400000 * 0x11111111
+// (mod 2^32) -- integer multiply-adds, which run on the FMA pipe and leave the ALU pipe (byte
+// permutes, logic, comparisons) to the rest of the quantizer.
 __device__ __forceinline__ uint32_t pack8_low_bytes(const uint32_t* k)
 {
-    const uint32_t even = prmt(prmt(k[0], k[2], 0x0040u), prmt(k[4], k[6], 0x0040u), 0x5410u);
-    const uint32_t odd = prmt(prmt(k[1], k[3], 0x0040u), prmt(k[5], k[7], 0x0040u), 0x5410u);
-    return even | (odd << 4);
+    uint32_t acc = k[0] + 0xC0C00000u;  // -(0x4B400000 * 0x11111111) mod 2^32
+#pragma unroll
+    for (int j = 1; j < 8; ++j) acc += k[j] << (4 * j);
+    return acc;
 }
 
 // E2M1 sign bits (bit 4j + 3) of the 8 bf16 values of a 16-byte vector.  A prmt selector

@@ -275,17 +275,22 @@ __global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
 }
 
 // ------------------------------------------------------------------------------------------
-// Pass 2b: tile quantizer.  A CTA stages a 64-row x 128-column tile in shared memory (rows
-// padded to 136 elements so both the row and the column walks are free of bank conflicts)
-// and produces
+// Pass 2b: tile quantizer.  A CTA stages 64-row x 128-column tiles in shared memory (rows
+// padded to 136 elements so that neither walk has bank conflicts), two buffers deep: while one
+// tile is quantized, the next one's rows are already being copied in (cp.async, 16 bytes per
+// copy, zero-filled outside the matrix).  Each tile gives
 //   ROW: the row-wise output (blocks along the columns), thread t -> row t % 64, blocks
 //        4 (t / 64) .. +3: 32 contiguous code bytes and one scale word;
 //   COL: the column-wise output (x^T, blocks along the rows, optionally RHT'd), thread t ->
-//        column t, the tile's 4 row blocks: 32 contiguous code bytes and one scale word.
+//        the column pair 2 (t % 64), 2 (t % 64) + 1 and rows 32 (t / 64) .. +31 (two blocks):
+//        one 32-bit shared load brings a row's values of both columns, the Hadamard sign of
+//        that row flips both with one xor on the packed pair; per column 16 code bytes and two
+//        scale bytes.
 // BLOCK2D: the scale of every 16x16 sub-tile comes from its maximum, shared by both outputs,
 // whose codes are then the same nibbles transposed.
 // ------------------------------------------------------------------------------------------
 constexpr int kTileRows = 64, kTileCols = 128, kTilePitch = 136;
+constexpr int kTileElems = kTileRows * kTilePitch;
 
 template <bool SR>
 __device__ __forceinline__ void encode16(const float* y, const BlockScale& bs, const Philox& ph,
@@ -309,10 +314,57 @@ __device__ __forceinline__ void encode16(const float* y, const BlockScale& bs, c
     w1 = p[1];
 }
 
-template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
-__global__ void __launch_bounds__(128, SR ? 6 : 8) quant_tile_kernel(TileArgs a)
+// Queue the copies of one tile's rows into `buf` (cp.async, 16 bytes each, zero-filled for
+// rows or column chunks outside the matrix) as one commit group.
+__device__ __forceinline__ void tile_load_async(const TileArgs& a, uint16_t* buf, int64_t r0,
+                                                int64_t c0, int nr, int nc)
 {
-    __shared__ __align__(16) uint16_t tile[kTileRows * kTilePitch];
+    const int t = threadIdx.x;
+    const uint32_t base = static_cast<uint32_t>(__cvta_generic_to_shared(buf));
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int ch = t + 128 * k, row = ch >> 4, cc = ch & 15;
+        const bool in = row < nr && cc * 8 < nc;
+        const uint16_t* src = in ? a.x + (r0 + row) * a.ld + c0 + cc * 8 : a.x;
+        const uint32_t dst = base + 2u * static_cast<uint32_t>(row * kTilePitch + cc * 8);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                     "r"(in ? 16 : 0)
+                     : "memory");
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// y = (1/4) H x over 16 values whose random signs are already applied: Sylvester butterflies of
+// widths 1, 2, 4, 8, then the exact scaling by 1/4 -- rht16 without its sign step.
+__device__ __forceinline__ void rht16_presigned(float* v)
+{
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i & h) continue;
+            const float a = v[i], b = v[i + h];
+            v[i] = __fadd_rn(a, b);
+            v[i + h] = __fsub_rn(a, b);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
+}
+
+// CTAs per SM: the stochastic-rounding variants are bound by instruction issue and trade
+// registers for resident warps differently (B200: the one-output RHT + SR pass is fastest with
+// 4 CTAs of 128 registers, the two-output pass with 6 of 80).
+template <bool ROW, bool COL, bool SR>
+constexpr int tile_ctas_per_sm()
+{
+    return SR && !(ROW && COL) ? 4 : 6;
+}
+
+template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
+__global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant_tile_kernel(TileArgs a)
+{
+    __shared__ __align__(16) uint16_t tiles[2 * kTileElems];
     __shared__ float bmax[kTileRows][8];
     __shared__ float tmax[4][8];
 
@@ -331,28 +383,48 @@ __global__ void __launch_bounds__(128, SR ? 6 : 8) quant_tile_kernel(TileArgs a)
     __shared__ float r_tab_row[128], r_tab_col[128];
     fill_factor_table(r_tab_row, ts_row.s_enc);
     fill_factor_table(r_tab_col, ts_col.s_enc);
-    __syncthreads();
+    // the Hadamard signs as xor masks on a packed bf16 pair (row i of a block: bit i)
+    uint32_t flip2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) flip2[i] = ((a.sign_mask >> i) & 1u) ? 0x80008000u : 0u;
     const Philox philox{a.keys};
     const int t = threadIdx.x;
     const int64_t tiles_c = (a.cols + kTileCols - 1) / kTileCols;
     const int64_t tiles_r = (a.rows + kTileRows - 1) / kTileRows;
     const int64_t ntiles = tiles_c * tiles_r;
-
-    for (int64_t id = blockIdx.x; id < ntiles; id += gridDim.x) {
-        const int64_t tid = ntiles - 1 - id;  // reverse order (L2 reuse)
-        const int64_t r0 = (tid / tiles_c) * kTileRows, c0 = (tid % tiles_c) * kTileCols;
-        const int nr = static_cast<int>(a.rows - r0 < kTileRows ? a.rows - r0 : kTileRows);
-        const int nc = static_cast<int>(a.cols - c0 < kTileCols ? a.cols - c0 : kTileCols);
-
-        __syncthreads();  // the previous tile's readers are done with `tile`
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const int ch = t + 128 * k, row = ch >> 4, cc = ch & 15;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (row < nr && cc * 8 < nc)
-                v = __ldg(reinterpret_cast<const uint4*>(a.x + (r0 + row) * a.ld + c0) + cc);
-            *reinterpret_cast<uint4*>(tile + row * kTilePitch + cc * 8) = v;
+    // tiles are visited in reverse order (the amax pass left the tensor's tail in L2)
+    auto coords = [&](int64_t id, int64_t& r0, int64_t& c0, int& nr, int& nc) {
+        const int64_t tid = ntiles - 1 - id;
+        r0 = (tid / tiles_c) * kTileRows;
+        c0 = (tid % tiles_c) * kTileCols;
+        nr = static_cast<int>(a.rows - r0 < kTileRows ? a.rows - r0 : kTileRows);
+        nc = static_cast<int>(a.cols - c0 < kTileCols ? a.cols - c0 : kTileCols);
+    };
+    {
+        int64_t r0, c0;
+        int nr, nc;
+        if (blockIdx.x < ntiles) {
+            coords(blockIdx.x, r0, c0, nr, nc);
+            tile_load_async(a, tiles, r0, c0, nr, nc);
         }
+    }
+    __syncthreads();  // the factor tables
+
+    int k = 0;
+    for (int64_t id = blockIdx.x; id < ntiles; id += gridDim.x, ++k) {
+        int64_t r0, c0;
+        int nr, nc;
+        coords(id, r0, c0, nr, nc);
+        const uint16_t* tile = tiles + (k & 1) * kTileElems;
+        if (id + gridDim.x < ntiles) {
+            int64_t r1, c1;
+            int nr1, nc1;
+            coords(id + gridDim.x, r1, c1, nr1, nc1);
+            tile_load_async(a, tiles + ((k + 1) & 1) * kTileElems, r1, c1, nr1, nc1);
+        } else {
+            asm volatile("cp.async.commit_group;" ::: "memory");  // keeps one group per tile
+        }
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's copies landed
         __syncthreads();
 
         // Row walk: thread t -> row t % 64, blocks 4 (t / 64) .. +3.  One 16-value block is
@@ -436,67 +508,87 @@ __global__ void __launch_bounds__(128, SR ? 6 : 8) quant_tile_kernel(TileArgs a)
                                          sf_offset(r, (c0 >> 4) + rblk, a.cols >> 6)) = sfw;
         }
 
-        if (COL && t < nc) {
-            const int64_t orow = c0 + t;  // output row = input column
-            uint32_t words[8];
-            uint32_t sfw = 0;
-            auto load_col_block = [&](int q, float* y) {
+        // Column walk: thread t -> columns 2p, 2p + 1 (p = t % 64), rows 32h .. 32h + 31
+        // (h = t / 64).  Rows are a multiple of 64 whenever column-wise output is asked for,
+        // so every tile has all 64 rows.
+        const int p = t & 63, h = t >> 6;
+        if (COL && 2 * p < nc) {
+            const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(tile) + p;
+            // y0 / y1: the 16 values of block q of the two columns (signs applied for RHT)
+            auto load_col_pair = [&](int q, float* y0, float* y1) {
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    y[i] = __uint_as_float(static_cast<uint32_t>(
-                               tile[(q * 16 + i) * kTilePitch + t]) << 16);
-                if (RHT) rht16(y, a.sign_mask);
+                for (int i = 0; i < 16; ++i) {
+                    uint32_t w = tile32[(32 * h + 16 * q + i) * (kTilePitch / 2)];
+                    if (RHT) w ^= flip2[i];
+                    y0[i] = bf16_lo(w);
+                    y1[i] = bf16_hi(w);
+                }
+                if (RHT) {
+                    rht16_presigned(y0);
+                    rht16_presigned(y1);
+                }
             };
+            uint32_t words[2][4];
+            uint32_t sfw[2] = {0u, 0u};
             if (MX) {
-                // 32-element blocks along the rows: the pairs (0, 1) and (2, 3) of 16-blocks
+                // one 32-element block per column: rows 32h .. 32h + 31
+                float y0[2][16], y1[2][16];
+                load_col_pair(0, y0[0], y1[0]);
+                load_col_pair(1, y0[1], y1[1]);
 #pragma unroll
-                for (int pr = 0; pr < 2; ++pr) {
-                    float y0[16], y1[16];
-                    load_col_block(2 * pr, y0);
-                    load_col_block(2 * pr + 1, y1);
+                for (int c = 0; c < 2; ++c) {
+                    float(*y)[16] = c ? y1 : y0;
                     float b = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) b = fmaxf(b, fmaxf(fabsf(y0[i]), fabsf(y1[i])));
+                    for (int i = 0; i < 16; ++i) b = fmaxf(b, fmaxf(fabsf(y[0][i]), fabsf(y[1][i])));
                     const BlockScale bs = mx_block_scale(b);
-                    const uint64_t e0 = static_cast<uint64_t>(orow) * a.rows + r0 + pr * 32;
-                    encode16<SR>(y0, bs, philox, e0, a.offset_col, words[4 * pr], words[4 * pr + 1]);
-                    encode16<SR>(y1, bs, philox, e0 + 16, a.offset_col, words[4 * pr + 2],
-                                 words[4 * pr + 3]);
-                    sfw |= (bs.sf | (bs.sf << 8)) << (16 * pr);
+                    const uint64_t e0 = static_cast<uint64_t>(c0 + 2 * p + c) * a.rows + r0 + 32 * h;
+                    encode16<SR>(y[0], bs, philox, e0, a.offset_col, words[c][0], words[c][1]);
+                    encode16<SR>(y[1], bs, philox, e0 + 16, a.offset_col, words[c][2],
+                                 words[c][3]);
+                    sfw[c] = bs.sf | (bs.sf << 8);
+                }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    float y0[16], y1[16];
+                    load_col_pair(q, y0, y1);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        const float* y = c ? y1 : y0;
+                        float b;
+                        if (BLOCK2D) {
+                            b = tmax[2 * h + q][(2 * p + c) >> 4];
+                        } else {
+                            b = 0.0f;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(y[i]));
+                        }
+                        const BlockScale bs = block_scale(b, ts_col.s_enc, r_tab_col);
+                        const uint64_t e0 =
+                            static_cast<uint64_t>(c0 + 2 * p + c) * a.rows + r0 + 32 * h + 16 * q;
+                        encode16<SR>(y, bs, philox, e0, a.offset_col, words[c][2 * q],
+                                     words[c][2 * q + 1]);
+                        sfw[c] |= bs.sf << (8 * q);
+                    }
                 }
             }
 #pragma unroll
-            for (int q = 0; q < (MX ? 0 : 4); ++q) {
-                float y[16];
+            for (int c = 0; c < 2; ++c) {
+                if (ts_col.nonfinite) {
+                    sfw[c] = 0;
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    y[i] = __uint_as_float(static_cast<uint32_t>(
-                               tile[(q * 16 + i) * kTilePitch + t]) << 16);
-                if (RHT) rht16(y, a.sign_mask);
-                float b;
-                if (BLOCK2D) {
-                    b = tmax[q][t >> 4];
-                } else {
-                    b = 0.0f;
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(y[i]));
+                    for (int q = 0; q < 4; ++q) words[c][q] = 0;
                 }
-                const BlockScale bs = block_scale(b, ts_col.s_enc, r_tab_col);
-                const uint64_t e0 = static_cast<uint64_t>(orow) * a.rows + r0 + q * 16;
-                encode16<SR>(y, bs, philox, e0, a.offset_col, words[2 * q], words[2 * q + 1]);
-                sfw |= bs.sf << (8 * q);
+                const int64_t orow = c0 + 2 * p + c;  // output row = input column
+                *reinterpret_cast<uint4*>(a.col_codes + (orow * a.rows + r0 + 32 * h) / 2) =
+                    make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]);
+                *reinterpret_cast<uint16_t*>(
+                    a.col_scales + sf_offset(orow, (r0 >> 4) + 2 * h, a.rows >> 6)) =
+                    static_cast<uint16_t>(sfw[c]);
             }
-            if (ts_col.nonfinite) {
-                sfw = 0;
-#pragma unroll
-                for (int q = 0; q < 8; ++q) words[q] = 0;
-            }
-            uint4* dst = reinterpret_cast<uint4*>(a.col_codes + (orow * a.rows + r0) / 2);
-            dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-            dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-            *reinterpret_cast<uint32_t*>(a.col_scales + sf_offset(orow, r0 >> 4, a.rows >> 6)) =
-                sfw;
         }
+        __syncthreads();  // everyone is done with this buffer before it is refilled
     }
     const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;

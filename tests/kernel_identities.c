@@ -50,19 +50,18 @@ int64_t kid_div6_mismatches(uint32_t lo, uint32_t hi, uint32_t* first_bad)
 }
 
 /* e2m1_sr_code: the magnitude code of a >= 0 stochastically rounded with the 16-bit random
- * integer r16, on the FMA pipe: the lines 2^17 a (exact), RU(2^16 a + 2^17), RU(2^15 a + 2^18)
- * and 7 * 2^16, their minimum m'; P = RU(m' + 2^23); Q = P - (2^23 + r16) (exact);
- * k = RU(Q 2^-16 + 1.5 * 2^23); the code is the low byte of k's pattern. */
+ * integer r16, on the FMA pipe: the lines 2^17 a, 2^16 a + 2^17 and 2^15 a + 2^18, each plus
+ * 2^23 and rounded upward by one FMA, and the constant 2^23 + 7 * 2^16; their minimum P;
+ * Q = P - (2^23 + r16) (exact); k = RU(Q 2^-16 + 1.5 * 2^23); the code is the low byte of k's
+ * pattern. */
 static uint32_t sr_code_emul(float a, uint32_t r16)
 {
     const float rbits = f_of(0x4B000000u | (r16 & 0xFFFFu)); /* 2^23 + r16 */
-    fesetround(FE_TONEAREST);
-    float l0 = a * 131072.0f;
     fesetround(FE_UPWARD);
-    float l1 = fmaf(a, 65536.0f, 131072.0f);
-    float l2 = fmaf(a, 32768.0f, 262144.0f);
-    float m = fminf(fminf(fminf(l0, l1), l2), 458752.0f);
-    float P = m + 8388608.0f;
+    float l0 = fmaf(a, 131072.0f, 8388608.0f);
+    float l1 = fmaf(a, 65536.0f, 8519680.0f);
+    float l2 = fmaf(a, 32768.0f, 8650752.0f);
+    float P = fminf(fminf(fminf(l0, l1), l2), 8847360.0f);
     fesetround(FE_TONEAREST);
     float Q = P - rbits;
     fesetround(FE_UPWARD);
