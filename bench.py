@@ -613,7 +613,18 @@ def run_kernel_case(args):
     T, D, F = 8192, 5120, 20480
     dev = torch.device("cuda", torch.cuda.current_device())
     ws = torch.empty((B.workspace_bytes(1 << 14, 1 << 14),), dtype=torch.uint8, device=dev)
-    if args.kernel in ("gemm", "gemm_amax", "chain", "chain_amax", "gemm_mx"):
+    if args.kernel == "gemm_f32":
+        # the wgrad GEMM of the MLP's up-projection: dW [20480 x 5120] = dY^T . X over K = 8192
+        # tokens, FP32 out, both operands RHT'd column-wise quantizations
+        dY = torch.from_numpy(synth.gradients((T, F), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
+        X = torch.from_numpy(synth.activations((T, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
+        qa = B.rht_quantize(dY, 0x5A3C, B.SR, seed=1, offset=1, workspace=ws)
+        qb = B.rht_quantize(X, 0x5A3C, 0, workspace=ws)
+        out = torch.empty((F, D), dtype=torch.float32, device=dev)
+        fn = lambda: B.gemm(qa, qb, out=out)  # noqa: E731
+        work, unit, peak = 2 * T * D * F / 1e12, "TFLOP/s", peaks["bf16_tflops"] * FP4_OVER_BF16
+        shape = f"M={F} N={D} K={T}, FP32 out"
+    elif args.kernel in ("gemm", "gemm_amax", "chain", "chain_amax", "gemm_mx"):
         X = torch.from_numpy(synth.activations((T, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
         W = torch.from_numpy(synth.weights((F, D), seed=2).view(np.int16)).view(torch.bfloat16).to(dev)
         mx = B.MX if args.kernel == "gemm_mx" else 0
@@ -650,9 +661,20 @@ def run_kernel_case(args):
         if args.kernel == "rowwise":
             q = B.QuantizedTensor(T, F, dev)
             fn = lambda: B.quantize(x, B.ROWWISE | B.SR, seed=1, out_row=q, workspace=ws)  # noqa: E731
+        elif args.kernel == "rowwise_rtn":
+            q = B.QuantizedTensor(T, F, dev)
+            fn = lambda: B.quantize(x, B.ROWWISE, out_row=q, workspace=ws)  # noqa: E731
         elif args.kernel == "tile2d":
-            q = B.QuantizedTensor(F, T, dev)
-            fn = lambda: B.quantize(x, B.COLWISE | B.BLOCK2D, out_col=q, workspace=ws)  # noqa: E731
+            # as the step quantizes W: 16x16 scales, row-wise and column-wise outputs
+            q = B.QuantizedTensor(T, F, dev)
+            q2 = B.QuantizedTensor(F, T, dev)
+            fn = lambda: B.quantize(x, B.ROWWISE | B.COLWISE | B.BLOCK2D, out_row=q,  # noqa: E731
+                                    out_col=q2, workspace=ws)
+        elif args.kernel == "dual_rtn":
+            q = B.QuantizedTensor(T, F, dev)
+            q2 = B.QuantizedTensor(F, T, dev)
+            fn = lambda: B.quantize_row_rht(x, 0x5A3C, 0, out_row=q, out_col=q2,  # noqa: E731
+                                            workspace=ws)
         elif args.kernel == "rht":
             q = B.QuantizedTensor(F, T, dev)
             fn = lambda: B.rht_quantize(x, 0x5A3C, B.SR, seed=1, out_col=q, workspace=ws)  # noqa: E731
@@ -668,7 +690,7 @@ def run_kernel_case(args):
             q2 = B.QuantizedTensor(F, T, dev)
             fn = lambda: B.quantize_row_rht(x, 0x5A3C, B.SR, seed=1, out_row=q, out_col=q2,  # noqa: E731
                                             workspace=ws)
-        outs = 2 if args.kernel == "dual" else 1
+        outs = 2 if args.kernel in ("dual", "dual_rtn", "tile2d") else 1
         work, unit, peak = n * (4 + outs * (0.5 + 1 / 16)) / 1e9, "GB/s", peaks["hbm_gbs"]
         shape = f"{T} x {F} bf16, amax pass + quantize pass"
     for _ in range(args.warmup):
@@ -841,9 +863,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["gemm", "gemm_amax", "chain", "chain_amax", "gemm_mx",
-                                         "rowwise", "tile2d", "rht", "dual", "rowwise_mx",
-                                         "rht_mx"], default=None,
+    ap.add_argument("--kernel", choices=["gemm", "gemm_f32", "gemm_amax", "chain", "chain_amax",
+                                         "gemm_mx", "rowwise", "rowwise_rtn", "tile2d", "rht",
+                                         "dual", "dual_rtn", "rowwise_mx", "rht_mx"], default=None,
                     help="time one kernel family alone at the workload's shapes (profiling)")
     ap.add_argument("--sweep", action="store_true",
                     help="quantizer bandwidth sweep over 2^n-element tensors (one line per point)")

@@ -8,20 +8,27 @@
 // 256 x 256 output tiles; each pair tile is one tcgen05.mma.cta_group::2 accumulation (M 256,
 // N 256, K 64 per instruction) whose A rows and B rows are split between the two CTAs, so each
 // SM reads 128 A rows and 128 B rows per K block: 38 KB per 256-wide K block where a single-CTA
-// 128 x 256 tile needs 54 KB for the same work.  22 warps per CTA:
+// 128 x 256 tile needs 54 KB for the same work.  23 warps per CTA:
 //   warp 0      TMA producer (both CTAs): per 256-wide K block, this CTA's A (128 x 128 B) and
 //               B (128 x 128 B) code boxes with 128-byte swizzle, this CTA's 128 rows of A
-//               scales and all 256 rows of B scales (contiguous 512-byte tiles of the MMA scale
-//               layout, bulk copies), into a shared-memory ring of 5 stages.
+//               scales (four 512-byte tiles of the MMA scale layout) and all 256 rows of B
+//               scales (eight), each set one 3-D tensor copy over the tiles, into a
+//               shared-memory ring of 5 stages.
 //   warps 2-5   scale stagers, one per 32-lane quarter of tensor memory (both CTAs): move each
 //               stage's scales shared -> registers -> tensor memory (tcgen05.st), then arrive on
 //               the leader CTA's stage barrier.  (tcgen05.cp from the MMA thread would use the
 //               tensor pipe: measured on B200, twelve 32x128b copies per K block lengthen the
 //               block's four MMAs from 278 ns to 458 ns.)
 //   warp 1      tensor-memory owner (both CTAs, allocated for the pair) and, in the leader CTA,
-//               the MMA issuer (one thread): once both CTAs' stagers have arrived, four
-//               kind::mxf4nvf4 block-scaled MMAs (E4M3 scales, or UE8M0 for MXFP4 operands),
-//               then one commit that releases the stage in both CTAs.
+//               the MMA issuer (one thread): per K block, four kind::mxf4nvf4 block-scaled MMAs
+//               (E4M3 scales, or UE8M0 for MXFP4 operands), then one commit that releases the
+//               stage in both CTAs.
+//   warp 22     the issuer's gate (leader CTA): waits until both CTAs' stagers have arrived
+//               (and, at a tile start, both epilogues have drained the accumulator), then
+//               meets the issuer at the slot's named barrier.  The issuer polls no mbarrier:
+//               measured on B200, a barrier poll in the issuing thread between two K blocks
+//               idles the tensor pipe 80-200 ns per K block (pair M256 N256 K64 MMAs:
+//               278 ns per four behind a named barrier, 480 ns with a commit and a poll).
 //   warps 6-21  epilogue (both CTAs): each warp drains one 32-lane quarter x 64 columns of its
 //               CTA's 128 x 256 half of the accumulator (tcgen05.ld), releases it to the leader,
 //               scales by 1 / (S_enc,A S_enc,B) and writes it while the next tile computes: bf16
@@ -63,7 +70,10 @@ constexpr int NUM_SF_WARPS = 4;         // one per 32-lane quarter of tensor mem
 constexpr int NUM_EPI_WARPS = 16;       // four per lane quarter, 64 accumulator columns each
 constexpr int FIRST_SF_WARP = 2;
 constexpr int FIRST_EPI_WARP = FIRST_SF_WARP + NUM_SF_WARPS;
-constexpr int THREADS = 32 * (FIRST_EPI_WARP + NUM_EPI_WARPS);
+constexpr int GATE_WARP = FIRST_EPI_WARP + NUM_EPI_WARPS;
+constexpr int THREADS = 32 * (GATE_WARP + 1);
+constexpr uint32_t GATE_BAR0 = 3;       // named barriers 3 .. 3 + STAGES - 1: issuer + gate
+constexpr uint32_t GATE_THREADS = 64;   // (1 and 2 are the epilogue's)
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;              // accumulator: columns [0, 256)
 constexpr int SF_COL = BN;              // scales: 48 columns per stage from column 256
@@ -669,16 +679,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 if (n_s) wait_bounded(bar(BAR_FULL + s), (n_s - 1) & 1, abort_flag, nullptr, true);
             }
         }
-    } else if (warp == 1 && lane == 0 && rank == 0) {
+    } else if (warp == 1 && rank == 0) {
         // ---------------- MMA issuer (leader CTA) ----------------
         // The MMA instructions issue at about the rate the tensor pipe executes them, so every
-        // instruction this thread runs between two K blocks leaves the pipe idle.  The loop is
-        // unrolled over the ring's slots, which it visits in order across tiles as the producer
-        // and the stagers do, so each slot's descriptors, scale columns and barriers are
-        // constants; the next slot's barrier is tested (and the fence taken) before this slot's
-        // last MMA, and the commit follows it.  Descriptors address shared memory through a
-        // 14-bit start-address field (address / 16): a slot is STAGE_BYTES / 16 further on, a K
-        // step 32 bytes (2 units).
+        // instruction this thread runs between two K blocks leaves the pipe idle.  The whole
+        // warp meets the gate warp at the slot's named barrier (the gate has seen the slot's
+        // operands and scales land); lane 0 then issues.  The loop is unrolled over the ring's
+        // slots, which it visits in order across tiles as the producer, the stagers and the
+        // gate do, so each slot's descriptors, scale columns, barriers and named barrier are
+        // constants.  Descriptors address shared memory through a 14-bit start-address field
+        // (address / 16): a slot is STAGE_BYTES / 16 further on, a K step 32 bytes (2 units).
+        // After an abort the gate keeps meeting the issuer, which then runs its schedule on
+        // stale operands (in bounds, results discarded) rather than leave a barrier unmet.
         const uint32_t s0 = smem_u32(smem);
         uint64_t da[STAGES], db[STAGES];
         uint32_t tc[STAGES];
@@ -690,62 +702,72 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         const uint32_t acc = tmem_base + ACC_COL;
         const bool k_full = (k_steps_total % (BK / MMA_K)) == 0;  // every stage has 4 K steps
-        uint32_t phase = 0;
-        bool ok = true, any = false;
-        int it = 0, kb = 0, t = cluster;
+        bool any = false;
+        int kb = 0, t = cluster;
         bool live = t < total;
-        while (live && ok) {
+        while (live) {
 #pragma unroll
             for (int j = 0; j < STAGES; ++j) {
-                if (!live || !ok) break;
-                if (kb == 0) {
-                    // tile start: both CTAs' epilogues have drained the previous accumulator,
-                    // and this slot's operands and scales are in place
-                    if (!wait_spin(bar(BAR_ACC_EMPTY), (it & 1) ^ 1, abort_flag, p.dev_status) ||
-                        !wait_bounded(bar(BAR_SF + j), phase, abort_flag, p.dev_status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                }
+                if (!live) break;
+                named_sync(GATE_BAR0 + j, GATE_THREADS);
                 const bool more = kb + 1 < num_kb;
-                const int jn = j + 1 == STAGES ? 0 : j + 1;
-                const uint32_t pn = j + 1 == STAGES ? phase ^ 1 : phase;
-                // K step k: scales of A in columns tc + 4k, of B in tc + 16 + 8k
-                if (k_full || more) {
-                    mma_nvf4_pair<MX>(acc, da[j], db[j], tc[j], tc[j] + 16, kb != 0 ? 1u : 0u);
-                    mma_nvf4_pair<MX>(acc, da[j] + 2, db[j] + 2, tc[j] + 4, tc[j] + 24, 1u);
-                    mma_nvf4_pair<MX>(acc, da[j] + 4, db[j] + 4, tc[j] + 8, tc[j] + 32, 1u);
-                    if (more) {
-                        if (!mbar_test_wait(bar(BAR_SF + jn), pn) &&
-                            !wait_bounded(bar(BAR_SF + jn), pn, abort_flag, p.dev_status))
-                            ok = false;
-                        tc_fence_after();
+                if (lane == 0) {
+                    tc_fence_after();
+                    // K step k: scales of A in columns tc + 4k, of B in tc + 16 + 8k
+                    if (k_full || more) {
+                        mma_nvf4_pair<MX>(acc, da[j], db[j], tc[j], tc[j] + 16, kb != 0 ? 1u : 0u);
+                        mma_nvf4_pair<MX>(acc, da[j] + 2, db[j] + 2, tc[j] + 4, tc[j] + 24, 1u);
+                        mma_nvf4_pair<MX>(acc, da[j] + 4, db[j] + 4, tc[j] + 8, tc[j] + 32, 1u);
+                        mma_nvf4_pair<MX>(acc, da[j] + 6, db[j] + 6, tc[j] + 12, tc[j] + 40, 1u);
+                    } else {
+                        const int nk = k_steps_total - kb * (BK / MMA_K);  // 1..3 K steps left
+                        for (int k = 0; k < nk; ++k)
+                            mma_nvf4_pair<MX>(acc, da[j] + 2 * k, db[j] + 2 * k, tc[j] + 4 * k,
+                                              tc[j] + 16 + 8 * k, (kb | k) != 0 ? 1u : 0u);
                     }
-                    mma_nvf4_pair<MX>(acc, da[j] + 6, db[j] + 6, tc[j] + 12, tc[j] + 40, 1u);
-                } else {
-                    const int nk = k_steps_total - kb * (BK / MMA_K);  // 1..3 K steps left
-                    for (int k = 0; k < nk; ++k)
-                        mma_nvf4_pair<MX>(acc, da[j] + 2 * k, db[j] + 2 * k, tc[j] + 4 * k,
-                                          tc[j] + 16 + 8 * k, (kb | k) != 0 ? 1u : 0u);
+                    mma_commit_pair(bar(BAR_EMPTY + j));
+                    if (!more) mma_commit_pair(bar(BAR_ACC_FULL));
                 }
+                __syncwarp();
                 any = true;
-                mma_commit_pair(bar(BAR_EMPTY + j));
                 if (!more) {
-                    if (ok) mma_commit_pair(bar(BAR_ACC_FULL));
                     kb = 0;
-                    ++it;
                     t += clusters;
                     live = t < total;
                 } else {
                     ++kb;
                 }
             }
-            phase ^= 1;
         }
-        if (!ok && any) {
+        // every MMA this CTA pair issued completes before the tensor memory can be freed
+        if (lane == 0 && any) {
             mma_commit_pair(bar(BAR_DRAIN));
             wait_bounded(bar(BAR_DRAIN), 0, abort_flag, nullptr, true);
+        }
+    } else if (warp == GATE_WARP && rank == 0) {
+        // ---------------- the issuer's gate (leader CTA) ----------------
+        // For each K block in the issuer's order: at a tile start, wait until both CTAs'
+        // epilogues have drained the accumulator; wait until both CTAs' stagers have put the
+        // slot's scales in tensor memory (which they do after the slot's TMA bytes landed);
+        // then meet the issuer.  After an abort (or a timeout here) it stops waiting but keeps
+        // meeting the issuer, K block for K block.
+        int stage = 0, it = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int t = cluster; t < total; t += clusters, ++it) {
+            for (int kb = 0; kb < num_kb; ++kb) {
+                if (lane == 0 && ok) {
+                    if (kb == 0)
+                        ok = wait_spin(bar(BAR_ACC_EMPTY), (it & 1) ^ 1, abort_flag, p.dev_status);
+                    if (ok) ok = wait_spin(bar(BAR_SF + stage), phase, abort_flag, p.dev_status);
+                }
+                __syncwarp();
+                named_sync(GATE_BAR0 + stage, GATE_THREADS);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1;
+                }
+            }
         }
     } else if (warp >= FIRST_SF_WARP && warp < FIRST_SF_WARP + NUM_SF_WARPS) {
         // ---------------- scale stagers (both CTAs) ----------------
