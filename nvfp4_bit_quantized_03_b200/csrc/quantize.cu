@@ -371,6 +371,10 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
     // Dual mode (row-wise output of x, column-wise output of RHT(x)): each output has its own
     // amax, hence its own tensor scale, and its own SR stream.  Otherwise one amax serves both.
     constexpr bool DUAL = ROW && COL && RHT;
+    // The SR pair inlines two Philox streams and two SR encoders per 16-value block; with its
+    // block loops unrolled the kernel body overflows the instruction cache ("no instruction"
+    // was its top stall), so those loops stay rolled.
+    constexpr bool kRollBlocks = DUAL && SR;
     TensorScale ts_row, ts_col;
     if (DUAL) {
         ts_row = fold_amax(a.src, a.row_amax, nullptr, a.dev_status);
@@ -459,7 +463,7 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
 
         if (ROW && rrow < nr && rblk * 16 < nc) {
             const int64_t r = r0 + rrow;
-            uint32_t words[8];
+            uint32_t words[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
             uint32_t sfw = 0;
             if (MX) {
                 // 32-element blocks: the pairs (0, 1) and (2, 3) of this thread's 16-blocks
@@ -479,7 +483,7 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
                     sfw |= (bs.sf | (bs.sf << 8)) << (16 * pr);
                 }
             }
-#pragma unroll
+#pragma unroll(kRollBlocks ? 1 : 4)
             for (int q = 0; q < (MX ? 0 : 4); ++q) {
                 float rv[16];
                 load_row_block(q, rv);
@@ -493,8 +497,15 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
                 }
                 const BlockScale bs = block_scale(b, ts_row.s_enc, r_tab_row);
                 const uint64_t e0 = static_cast<uint64_t>(r) * a.cols + c0 + (rblk + q) * 16;
-                encode16<SR>(rv, bs, philox, e0, a.offset, words[2 * q], words[2 * q + 1]);
-                sfw |= bs.sf << (8 * q);
+                uint32_t w0, w1;
+                encode16<SR>(rv, bs, philox, e0, a.offset, w0, w1);
+                // shift block q in at the top: after the loop block q sits in words 2q, 2q + 1
+                // and byte q of sfw (register moves only, also when the loop is not unrolled)
+#pragma unroll
+                for (int i = 0; i < 6; ++i) words[i] = words[i + 2];
+                words[6] = w0;
+                words[7] = w1;
+                sfw = (sfw >> 8) | (bs.sf << 24);
             }
             if (ts_row.nonfinite) {
                 sfw = 0;
@@ -528,7 +539,7 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
                     rht16_presigned(y1);
                 }
             };
-            uint32_t words[2][4];
+            uint32_t words[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
             uint32_t sfw[2] = {0u, 0u};
             if (MX) {
                 // one 32-element block per column: rows 32h .. 32h + 31
@@ -549,7 +560,7 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
                     sfw[c] = bs.sf | (bs.sf << 8);
                 }
             } else {
-#pragma unroll
+#pragma unroll(kRollBlocks ? 1 : 2)
                 for (int q = 0; q < 2; ++q) {
                     float y0[16], y1[16];
                     load_col_pair(q, y0, y1);
@@ -567,9 +578,14 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
                         const BlockScale bs = block_scale(b, ts_col.s_enc, r_tab_col);
                         const uint64_t e0 =
                             static_cast<uint64_t>(c0 + 2 * p + c) * a.rows + r0 + 32 * h + 16 * q;
-                        encode16<SR>(y, bs, philox, e0, a.offset_col, words[c][2 * q],
-                                     words[c][2 * q + 1]);
-                        sfw[c] |= bs.sf << (8 * q);
+                        uint32_t w0, w1;
+                        encode16<SR>(y, bs, philox, e0, a.offset_col, w0, w1);
+                        // block q ends in words[c][2q], [2q + 1] and byte q of sfw[c]
+                        words[c][0] = words[c][2];
+                        words[c][1] = words[c][3];
+                        words[c][2] = w0;
+                        words[c][3] = w1;
+                        sfw[c] = (sfw[c] >> 8) | (bs.sf << 8);
                     }
                 }
             }
