@@ -227,6 +227,54 @@ __device__ __forceinline__ float min3f(float a, float b, float c)
     return d;
 }
 
+// ---- paired FP32 lanes --------------------------------------------------------------------
+// sm_100 runs FP32 add, subtract, multiply and FMA on two lanes held in one 64-bit register
+// pair as one instruction (.f32x2).  Each lane is the IEEE operation with the stated rounding,
+// so pairing two independent operations halves their instruction count and changes no bit.
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float f2lo(uint64_t v)
+{
+    float lo;
+    asm("{\n\t.reg .f32 t;\n\tmov.b64 {%0, t}, %1;\n\t}" : "=f"(lo) : "l"(v));
+    return lo;
+}
+__device__ __forceinline__ float f2hi(uint64_t v)
+{
+    float hi;
+    asm("{\n\t.reg .f32 t;\n\tmov.b64 {t, %0}, %1;\n\t}" : "=f"(hi) : "l"(v));
+    return hi;
+}
+__device__ __forceinline__ uint64_t f2splat(float c) { return f2pack(c, c); }
+__device__ __forceinline__ uint64_t add2_rn(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t sub2_rn(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t mul2_rn(uint64_t a, uint64_t b)
+{
+    uint64_t d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma2_rp(uint64_t a, uint64_t b, uint64_t c)
+{
+    uint64_t d;
+    asm("fma.rp.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // Bit pattern of the FP32 value 2^23 + r16 for half h (0: low, 1: high) of a 32-bit random
 // word: the two bytes of the half under the exponent byte 0x4B.
 __device__ __forceinline__ uint32_t rand16_as_f32_bits(uint32_t word, int h)
@@ -244,6 +292,23 @@ __device__ __forceinline__ uint32_t e2m1_sr_code(float a, uint32_t rbits)
     const float P = fminf(min3f(l0, l1, l2), 8847360.0f);  // 2^23 + 7 * 2^16
     const float Q = __fsub_rn(P, __uint_as_float(rbits));
     return __float_as_uint(__fmaf_ru(Q, 0x1p-16f, 12582912.0f));
+}
+
+// e2m1_sr_code for two magnitudes at once, the two lanes of each FMA, subtraction and FMA
+// paired (the minima stay per lane).
+__device__ __forceinline__ void e2m1_sr_code2(float a0, float a1, uint32_t rb0, uint32_t rb1,
+                                              uint32_t& k0, uint32_t& k1)
+{
+    const uint64_t A = f2pack(a0, a1);
+    const uint64_t L0 = fma2_rp(A, f2splat(131072.0f), f2splat(8388608.0f));
+    const uint64_t L1 = fma2_rp(A, f2splat(65536.0f), f2splat(8519680.0f));
+    const uint64_t L2 = fma2_rp(A, f2splat(32768.0f), f2splat(8650752.0f));
+    const float P0 = fminf(min3f(f2lo(L0), f2lo(L1), f2lo(L2)), 8847360.0f);
+    const float P1 = fminf(min3f(f2hi(L0), f2hi(L1), f2hi(L2)), 8847360.0f);
+    const uint64_t Q = sub2_rn(f2pack(P0, P1), f2pack(__uint_as_float(rb0), __uint_as_float(rb1)));
+    const uint64_t K = fma2_rp(Q, f2splat(0x1p-16f), f2splat(12582912.0f));
+    k0 = __float_as_uint(f2lo(K));
+    k1 = __float_as_uint(f2hi(K));
 }
 
 // Eight codes from the patterns k[j] = 0x4B400000 + code_j packed as nibbles, element j at
@@ -290,9 +355,29 @@ __device__ __forceinline__ uint32_t e2m1x8_sr(const float* x, float r, const uin
     uint32_t k[8];
     const uint32_t w[4] = {rnd.x, rnd.y, rnd.z, rnd.w};
 #pragma unroll
-    for (int j = 0; j < 8; ++j)
-        k[j] = e2m1_sr_code(__fmul_rn(fabsf(x[j]), r), rand16_as_f32_bits(w[j >> 1], j & 1));
+    for (int j = 0; j < 8; j += 2)
+        e2m1_sr_code2(__fmul_rn(fabsf(x[j]), r), __fmul_rn(fabsf(x[j + 1]), r),
+                      rand16_as_f32_bits(w[j >> 1], 0), rand16_as_f32_bits(w[j >> 1], 1), k[j],
+                      k[j + 1]);
     return pack8_low_bytes(k) | signs;
+}
+
+// e2m1x8_sr of two independent groups of 8 (values, factor, random words, signs) in step, the
+// element j of both groups sharing paired lanes.
+__device__ __forceinline__ void e2m1x8_sr2(const float* xa, const float* xb, float ra, float rb,
+                                           const uint4& rnda, const uint4& rndb, uint32_t signsa,
+                                           uint32_t signsb, uint32_t& pa, uint32_t& pb)
+{
+    uint32_t ka[8], kb[8];
+    const uint32_t wa[4] = {rnda.x, rnda.y, rnda.z, rnda.w};
+    const uint32_t wb[4] = {rndb.x, rndb.y, rndb.z, rndb.w};
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        e2m1_sr_code2(__fmul_rn(fabsf(xa[j]), ra), __fmul_rn(fabsf(xb[j]), rb),
+                      rand16_as_f32_bits(wa[j >> 1], j & 1), rand16_as_f32_bits(wb[j >> 1], j & 1),
+                      ka[j], kb[j]);
+    pa = pack8_low_bytes(ka) | signsa;
+    pb = pack8_low_bytes(kb) | signsb;
 }
 
 // ---- random Hadamard transform ----------------------------------------------------------

@@ -185,9 +185,12 @@ __device__ __forceinline__ uint32_t encode8(const uint4& v, const float* e, cons
 {
     if (SR) return e2m1x8_sr(e, bs.r, ph.group(f, offset), signs8_bf16(v));
     uint32_t packed = 0;
+    const uint64_t r2 = f2splat(bs.r);
 #pragma unroll
-    for (int j = 0; j < 8; j += 2)
-        packed |= e2m1x2_rn(__fmul_rn(e[j], bs.r), __fmul_rn(e[j + 1], bs.r)) << (4 * j);
+    for (int j = 0; j < 8; j += 2) {
+        const uint64_t s2 = mul2_rn(f2pack(e[j], e[j + 1]), r2);
+        packed |= e2m1x2_rn(f2lo(s2), f2hi(s2)) << (4 * j);
+    }
     return packed;
 }
 
@@ -297,17 +300,20 @@ __device__ __forceinline__ void encode16(const float* y, const BlockScale& bs, c
                                          uint64_t e0, uint64_t offset, uint32_t& w0,
                                          uint32_t& w1)
 {
+    if (SR) {
+        // the block's two groups of 8 (one Philox call each) in step on paired lanes
+        e2m1x8_sr2(y, y + 8, bs.r, bs.r, ph.group(e0 >> 3, offset),
+                   ph.group((e0 >> 3) + 1, offset), signs8_f32(y), signs8_f32(y + 8), w0, w1);
+        return;
+    }
     uint32_t p[2] = {0u, 0u};
+    const uint64_t r2 = f2splat(bs.r);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        if (SR) {
-            p[h] = e2m1x8_sr(y + 8 * h, bs.r, ph.group((e0 >> 3) + h, offset),
-                             signs8_f32(y + 8 * h));
-        } else {
 #pragma unroll
-            for (int j = 0; j < 8; j += 2)
-                p[h] |= e2m1x2_rn(__fmul_rn(y[8 * h + j], bs.r), __fmul_rn(y[8 * h + j + 1], bs.r))
-                        << (4 * j);
+        for (int j = 0; j < 8; j += 2) {
+            const uint64_t s2 = mul2_rn(f2pack(y[8 * h + j], y[8 * h + j + 1]), r2);
+            p[h] |= e2m1x2_rn(f2lo(s2), f2hi(s2)) << (4 * j);
         }
     }
     w0 = p[0];
@@ -352,13 +358,31 @@ __device__ __forceinline__ void rht16_presigned(float* v)
     for (int i = 0; i < 16; ++i) v[i] = __fmul_rn(v[i], 0.25f);
 }
 
-// CTAs per SM: the stochastic-rounding variants are bound by instruction issue and trade
-// registers for resident warps differently (B200: the one-output RHT + SR pass is fastest with
-// 4 CTAs of 128 registers, the two-output pass with 6 of 80).
+// The same for two columns at once, column 0 in the low lane of each paired FP32 register.
+__device__ __forceinline__ void rht16_presigned2(uint64_t* v)
+{
+#pragma unroll
+    for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (i & h) continue;
+            const uint64_t a = v[i], b = v[i + h];
+            v[i] = add2_rn(a, b);
+            v[i + h] = sub2_rn(a, b);
+        }
+    }
+    const uint64_t quarter = f2splat(0.25f);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = mul2_rn(v[i], quarter);
+}
+
+// CTAs per SM: the stochastic-rounding variants are bound by instruction issue and run fastest
+// with 4 CTAs of up to 128 registers (B200, 8192 x 20480: the one-pass SR pair 0.425 ms
+// against 0.452 with 5 CTAs and 0.476 with 6, where it spills), the RTN ones with 6 of 80.
 template <bool ROW, bool COL, bool SR>
 constexpr int tile_ctas_per_sm()
 {
-    return SR && !(ROW && COL) ? 4 : 6;
+    return SR ? 4 : 6;
 }
 
 template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
@@ -526,17 +550,34 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
         if (COL && 2 * p < nc) {
             const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(tile) + p;
             // y0 / y1: the 16 values of block q of the two columns (signs applied for RHT)
+            // (SR variants, bound by instruction issue, run the two columns' butterflies on
+            // paired lanes; the RTN ones keep them per lane, which needs fewer registers)
             auto load_col_pair = [&](int q, float* y0, float* y1) {
+                if (RHT && SR) {
+                    uint64_t yy[16];  // row i of the block: (column 2p, column 2p + 1)
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    uint32_t w = tile32[(32 * h + 16 * q + i) * (kTilePitch / 2)];
-                    if (RHT) w ^= flip2[i];
-                    y0[i] = bf16_lo(w);
-                    y1[i] = bf16_hi(w);
-                }
-                if (RHT) {
-                    rht16_presigned(y0);
-                    rht16_presigned(y1);
+                    for (int i = 0; i < 16; ++i) {
+                        const uint32_t w = tile32[(32 * h + 16 * q + i) * (kTilePitch / 2)] ^ flip2[i];
+                        yy[i] = f2pack(bf16_lo(w), bf16_hi(w));
+                    }
+                    rht16_presigned2(yy);
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        y0[i] = f2lo(yy[i]);
+                        y1[i] = f2hi(yy[i]);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        uint32_t w = tile32[(32 * h + 16 * q + i) * (kTilePitch / 2)];
+                        if (RHT) w ^= flip2[i];
+                        y0[i] = bf16_lo(w);
+                        y1[i] = bf16_hi(w);
+                    }
+                    if (RHT) {
+                        rht16_presigned(y0);
+                        rht16_presigned(y1);
+                    }
                 }
             };
             uint32_t words[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
