@@ -92,26 +92,29 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
             for (int k = 0; k < 16; ++k)
                 mp = __vmaxu2(mp, __vmaxu2(v[k].x & 0x7FFF7FFFu, v[k].y & 0x7FFF7FFFu));
         }
+        // two columns per transform pass, on paired FP32 lanes (the packed bf16 pair of a word)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            float y[16];
+        for (int jp = 0; jp < 2; ++jp) {
+            uint64_t y[16];
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
-                const uint32_t w = (j < 2 ? v[k].x : v[k].y) ^ flip[k];
-                y[k] = (j & 1) ? bf16_hi(w) : bf16_lo(w);
+                const uint32_t w = (jp == 0 ? v[k].x : v[k].y) ^ flip[k];
+                y[k] = f2pack(bf16_lo(w), bf16_hi(w));
             }
 #pragma unroll
             for (int h = 1; h < 16; h <<= 1) {
 #pragma unroll
                 for (int k = 0; k < 16; ++k) {
                     if (k & h) continue;
-                    const float a = y[k], b = y[k + h];
-                    y[k] = __fadd_rn(a, b);
-                    y[k + h] = __fsub_rn(a, b);
+                    const uint64_t a = y[k], b = y[k + h];
+                    y[k] = add2_rn(a, b);
+                    y[k + h] = sub2_rn(a, b);
                 }
             }
 #pragma unroll
-            for (int k = 0; k < 16; ++k) m = max(m, __float_as_uint(y[k]) & 0x7FFFFFFFu);
+            for (int k = 0; k < 16; ++k)
+                m = max(m, max(__float_as_uint(f2lo(y[k])) & 0x7FFFFFFFu,
+                               __float_as_uint(f2hi(y[k])) & 0x7FFFFFFFu));
         }
     }
     // x1/4 of the largest magnitude (NaN and Inf stay at or above the Inf pattern)
