@@ -73,7 +73,7 @@ constexpr int FIRST_EPI_WARP = FIRST_SF_WARP + NUM_SF_WARPS;
 constexpr int GATE_WARP = FIRST_EPI_WARP + NUM_EPI_WARPS;
 constexpr int THREADS = 32 * (GATE_WARP + 1);
 constexpr uint32_t GATE_BAR0 = 3;       // named barriers 3 .. 3 + STAGES - 1: issuer + gate
-constexpr uint32_t GATE_THREADS = 64;   // (1 and 2 are the epilogue's)
+constexpr uint32_t GATE_THREADS = 64;   // (1 is the epilogue's)
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_COL = 0;              // accumulator: columns [0, 256)
 constexpr int SF_COL = BN;              // scales: 48 columns per stage from column 256
@@ -610,7 +610,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_init(bar(BAR_SF + s), 2 * NUM_SF_WARPS);
         }
         mbar_init(bar(BAR_ACC_FULL), 1);
-        mbar_init(bar(BAR_ACC_EMPTY), 2);  // one arrival per CTA's epilogue
+        mbar_init(bar(BAR_ACC_EMPTY), 2 * NUM_EPI_WARPS);  // every epilogue warp of the pair
         mbar_init(bar(BAR_DRAIN), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -862,9 +862,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             tmem_wait_ld();
             tc_fence_before();
-            // every epilogue warp holds its slice: one arrival releases the accumulator
-            named_sync(2, EPI_THREADS);
-            if (waiter) mbar_arrive_cluster(bar(BAR_ACC_EMPTY), 0);
+            // this warp holds its slice: its arrival releases its part of the accumulator
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(bar(BAR_ACC_EMPTY), 0);
 
             int tm, tn;
             tile_coords(t, tiles_m, tiles_n, tm, tn);
