@@ -388,10 +388,28 @@ constexpr int tile_ctas_per_sm()
     return SR ? 4 : 6;
 }
 
-template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
-__global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant_tile_kernel(TileArgs a)
+// Tile buffers per CTA.  Two (the next tile's copies in flight while this one is quantized),
+// except for the plain column-wise NVFP4 RTN passes (no RHT, no 16x16 scaling): they do little
+// arithmetic per byte, and one buffer halves their shared memory so that 8 CTAs share an SM,
+// which keeps more of HBM's latency covered (B200, 2^30 elements in rows of 4096: 0.976 ms
+// with one buffer and 8 CTAs against 1.10 ms with two buffers and 6).
+template <bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
+constexpr int tile_buffers()
 {
-    __shared__ __align__(16) uint16_t tiles[2 * kTileElems];
+    return COL && !BLOCK2D && !RHT && !SR && !MX ? 1 : 2;
+}
+template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
+constexpr int tile_min_ctas()
+{
+    return tile_buffers<COL, BLOCK2D, RHT, SR, MX>() == 1 ? 8 : tile_ctas_per_sm<ROW, COL, SR>();
+}
+
+template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
+__global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR, MX>()))
+    quant_tile_kernel(TileArgs a)
+{
+    constexpr int kBuffers = tile_buffers<COL, BLOCK2D, RHT, SR, MX>();
+    __shared__ __align__(16) uint16_t tiles[kBuffers * kTileElems];
     __shared__ float bmax[kTileRows][8];
     __shared__ float tmax[4][8];
 
@@ -434,7 +452,7 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
     {
         int64_t r0, c0;
         int nr, nc;
-        if (blockIdx.x < ntiles) {
+        if (kBuffers == 2 && blockIdx.x < ntiles) {
             coords(blockIdx.x, r0, c0, nr, nc);
             tile_load_async(a, tiles, r0, c0, nr, nc);
         }
@@ -446,16 +464,21 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
         int64_t r0, c0;
         int nr, nc;
         coords(id, r0, c0, nr, nc);
-        const uint16_t* tile = tiles + (k & 1) * kTileElems;
-        if (id + gridDim.x < ntiles) {
-            int64_t r1, c1;
-            int nr1, nc1;
-            coords(id + gridDim.x, r1, c1, nr1, nc1);
-            tile_load_async(a, tiles + ((k + 1) & 1) * kTileElems, r1, c1, nr1, nc1);
+        const uint16_t* tile = tiles + (kBuffers == 2 ? (k & 1) * kTileElems : 0);
+        if (kBuffers == 1) {
+            tile_load_async(a, tiles, r0, c0, nr, nc);
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         } else {
-            asm volatile("cp.async.commit_group;" ::: "memory");  // keeps one group per tile
+            if (id + gridDim.x < ntiles) {
+                int64_t r1, c1;
+                int nr1, nc1;
+                coords(id + gridDim.x, r1, c1, nr1, nc1);
+                tile_load_async(a, tiles + ((k + 1) & 1) * kTileElems, r1, c1, nr1, nc1);
+            } else {
+                asm volatile("cp.async.commit_group;" ::: "memory");  // keeps one group per tile
+            }
+            asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's copies landed
         }
-        asm volatile("cp.async.wait_group 1;" ::: "memory");  // this tile's copies landed
         __syncthreads();
 
         // Row walk: thread t -> row t % 64, blocks 4 (t / 64) .. +3.  One 16-value block is
@@ -546,11 +569,45 @@ __global__ void __launch_bounds__(128, (tile_ctas_per_sm<ROW, COL, SR>())) quant
                                          sf_offset(r, (c0 >> 4) + rblk, a.cols >> 6)) = sfw;
         }
 
-        // Column walk: thread t -> columns 2p, 2p + 1 (p = t % 64), rows 32h .. 32h + 31
-        // (h = t / 64).  Rows are a multiple of 64 whenever column-wise output is asked for,
-        // so every tile has all 64 rows.
+        // Column walks.  Rows are a multiple of 64 whenever column-wise output is asked for, so
+        // every tile has all 64 rows.
+        //  * The plain RTN pass (one buffer): thread t -> column t, all 64 rows (four blocks),
+        //    one 16-bit shared load per value; it writes 32 contiguous code bytes (a whole
+        //    sector) and one scale word per output row.
+        //  * Otherwise: thread t -> columns 2p, 2p + 1 (p = t % 64), rows 32h .. 32h + 31
+        //    (h = t / 64); one 32-bit shared load brings a row's values of both columns.
         const int p = t & 63, h = t >> 6;
-        if (COL && 2 * p < nc) {
+        if (kBuffers == 1) {
+            if (COL && t < nc) {
+                const int64_t orow = c0 + t;  // output row = input column
+                uint32_t words[8];
+                uint32_t sfw = 0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float y[16];
+                    float b = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        y[i] = __uint_as_float(
+                            static_cast<uint32_t>(tile[(16 * q + i) * kTilePitch + t]) << 16);
+                        b = fmaxf(b, fabsf(y[i]));
+                    }
+                    const BlockScale bs = block_scale(b, ts_col.s_enc, r_tab_col);
+                    encode16<false>(y, bs, philox, 0, 0, words[2 * q], words[2 * q + 1]);
+                    sfw |= bs.sf << (8 * q);
+                }
+                if (ts_col.nonfinite) {
+                    sfw = 0;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) words[q] = 0;
+                }
+                uint4* dst = reinterpret_cast<uint4*>(a.col_codes + (orow * a.rows + r0) / 2);
+                dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
+                dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
+                *reinterpret_cast<uint32_t*>(a.col_scales +
+                                             sf_offset(orow, r0 >> 4, a.rows >> 6)) = sfw;
+            }
+        } else if (COL && 2 * p < nc) {
             const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(tile) + p;
             // y0 / y1: the 16 values of block q of the two columns (signs applied for RHT)
             // (SR variants, bound by instruction issue, run the two columns' butterflies on
