@@ -31,9 +31,9 @@
 //               278 ns per four behind a named barrier, 480 ns with a commit and a poll).
 //   warps 6-21  epilogue (both CTAs): each warp drains one 32-lane quarter x 64 columns of its
 //               CTA's 128 x 256 half of the accumulator (tcgen05.ld), releases it to the leader,
-//               scales by 1 / (S_enc,A S_enc,B) and writes it while the next tile computes: bf16
-//               rows through a 512-byte per-warp staging buffer with paced TMA bulk tensor
-//               stores (clipped at the matrix edge), FP32 pairs straight from registers.  With
+//               scales by 1 / (S_enc,A S_enc,B) and writes it while the next tile computes,
+//               through a 2 KB per-warp staging buffer with TMA bulk tensor stores (2 rounds for
+//               bf16, 4 for FP32; clipped at the matrix edge).  With
 //               the fused amax, the bf16 epilogue also reduces max |D| and, by 16-lane shuffles
 //               across rows, max |RHT(D)| for the next quantization of D.
 // No load is multicast: every CTA loads its own operands from this GPU's memory.
@@ -80,18 +80,20 @@ constexpr int SF_COL = BN;              // scales: 48 columns per stage from col
 constexpr int SF_COLS_PER_STAGE = (BK / MMA_K) * (4 + 8);
 constexpr int BAR_BYTES = 256;
 
-// Pipeline shape per output type.  Five operand stages either way: a bf16 tile (64 KB of
-// output per CTA) goes out through 512-byte staging buffers with paced TMA stores (a
-// first-round delay and a gap between rounds, so that they do not crowd the next tile's first
-// operand loads); an FP32 tile (128 KB per CTA) is stored straight from registers.
+// Pipeline shape per output type.  Five operand stages either way.  A tile's output (64 KB per
+// CTA in bf16, 128 KB in FP32) goes out through a 2 KB staging buffer per epilogue warp: TMA
+// store rounds of 32 rows x 64 bytes, two for bf16 and four for FP32.  (With 512-byte buffers,
+// eight bf16 rounds whose store round trips follow one another bounded the epilogue: B200,
+// 8192 x 20480 x K, 0.421 -> 0.365 ms at K = 5120 and 0.322 -> 0.114 ms at K = 1024; delays
+// that paced the small rounds away from the next tile's loads no longer help.  FP32 rows
+// stored straight from registers were slower than the staged boxes: 0.387 against 0.375 ms at
+// 20480 x 5120 x 8192, 0.200 against 0.146 ms at 8192 x 20480 x 1024.)
 template <bool BF16>
 struct Pipe {
     static constexpr int STAGES = 5;
-    static constexpr int STAGING_BYTES = 512;  // per epilogue warp (bf16 boxes; FP32 stores direct)
+    static constexpr int STAGING_BYTES = 2048;  // per epilogue warp
     static constexpr int SMEM_BYTES =
         STAGES * STAGE_BYTES + NUM_EPI_WARPS * STAGING_BYTES + BAR_BYTES + 1024;
-    static constexpr unsigned FIRST_NS = BF16 ? 3000u : 0u;
-    static constexpr unsigned GAP_NS = BF16 ? 1000u : 2000u;
     // shared-memory barrier slots (the same offsets in both CTAs of a pair)
     static constexpr int BAR_FULL = 0;                     // [STAGES] this CTA's TMA bytes landed
     static constexpr int BAR_EMPTY = BAR_FULL + STAGES;    // [STAGES] the stage's MMAs completed
@@ -376,24 +378,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* v)
           "=r"(v[31])
         : "r"(taddr));
 }
-// 16 TMEM lanes x 8 groups of 8 FP32 columns: thread t receives, for group g, registers
-// v[4g], v[4g+1] = lane t / 4, columns 8g + 2 (t % 4) + {0, 1}, and v[4g+2], v[4g+3] = the
-// same columns of lane t / 4 + 8 (the 16x256b pattern, repeated 8 times along the columns).
-__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t* v)
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.16x256b.x8.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-        "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, "
-        "[%32];"
-        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
-          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
-          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
-          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
-          "=r"(v[31])
-        : "r"(taddr));
-}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Tensor encode scale of an operand, as the quantizer computed it; see Alpha below.
@@ -464,13 +448,11 @@ __device__ __forceinline__ void tile_coords(int t, int tiles_m, int tiles_n, int
 // One epilogue warp's 32 x 64 slice of the tile (row `lane`, values v[0..63] in FP32 bits) to
 // global memory, scaled by alpha and converted, through the warp's staging buffer with TMA bulk
 // tensor stores.
-//  * bf16: 8 rounds of 16 bytes (8 columns) of every row, boxes of 32 rows x 16 bytes; row
-//    `lane` of a box sits at lane * 16, so the warp's 16-byte shared stores are conflict-free.
-//  * FP32: 4 rounds of 64 bytes (16 columns), boxes of 32 rows x 64 bytes; row `lane` sits at
-//    lane * 64 with its four 16-byte chunks permuted by the 64-byte swizzle (chunk c at
-//    c ^ ((row / 2) % 4)), which the tensor map undoes.
-// Each round waits only for the previous box to leave the buffer; rounds are paced by
-// Pipe::FIRST_NS / GAP_NS.
+//  * bf16: 2 rounds of 64 bytes (32 columns) of every row; FP32: 4 rounds of 64 bytes
+//    (16 columns).  Boxes of 32 rows x 64 bytes: row `lane` sits at lane * 64 with its four
+//    16-byte chunks permuted by the 64-byte swizzle (chunk c at c ^ ((row / 2) % 4)), which
+//    keeps the warp's 16-byte shared stores conflict-free and which the tensor map undoes.
+// Each round waits only for the previous box to leave the buffer.
 // With AMAX (bf16 only) the warp also folds its slice into the two maxima the next quantizer
 // of D needs: m_plain, the largest |bf16| bit pattern (in the low 16 bits of each half), and
 // m_rht, the largest |v| bit pattern of the random Hadamard transform of every 16 consecutive
@@ -484,15 +466,12 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, const Alpha& alph
                                             int M, int N, uint32_t* m_plain = nullptr,
                                             uint32_t* m_rht = nullptr, uint32_t flip = 0)
 {
-    using P = Pipe<BF16>;
-    constexpr int CHUNKS = BF16 ? 1 : 4;             // 16-byte chunks per box row
+    constexpr int CHUNKS = 4;                        // 16-byte chunks per box row
     constexpr int COLS = CHUNKS * (BF16 ? 8 : 4);    // columns per box row
     const uint32_t row_base = stage_buf + 16 * CHUNKS * lane;
-    const uint32_t swz = BF16 ? 0u : ((lane >> 1) & 3);
+    const uint32_t swz = (lane >> 1) & 3;
 #pragma unroll
     for (int r = 0; r < 64 / COLS; ++r) {
-        if (r == 0 && P::FIRST_NS) __nanosleep(P::FIRST_NS);
-        if (r != 0 && P::GAP_NS) __nanosleep(P::GAP_NS);
         if (lane == 0) bulk_wait_read();  // the previous box has left the buffer
         __syncwarp();
 #pragma unroll
@@ -501,7 +480,7 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, const Alpha& alph
             if (BF16) {
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
-                    const int j = r * 8 + 2 * h;
+                    const int j = r * COLS + c * 8 + 2 * h;
                     const __nv_bfloat162 b2 =
                         __floats2bfloat162_rn(apply_alpha(v[j], alpha), apply_alpha(v[j + 1], alpha));
                     o[h] = *reinterpret_cast<const uint32_t*>(&b2);
@@ -540,33 +519,6 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, const Alpha& alph
         __syncwarp();
         const int x = n0 + r * COLS;
         if (lane == 0 && y < M && x < N) tma_store_2d(tmap_d, stage_buf, x, y);
-    }
-}
-
-// One epilogue warp's 32 x 64 FP32 slice straight from registers (the 16x256b layout of
-// tmem_ld_16x256b_x8 for the two 16-row halves): scaled by alpha, each instruction writes 8 B
-// per thread, i.e. 8 rows x 32 contiguous bytes (whole sectors) per warp; no staging, so the
-// FP32 kernel keeps the shared memory for operand stages like the bf16 one.
-__device__ __forceinline__ void store_f32_direct(const uint32_t* v, const Alpha& alpha, float* D,
-                                                 int64_t ldd, int lane, int n0, int y, int M,
-                                                 int N)
-{
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            const int col = n0 + 8 * g + 2 * (lane & 3);
-            const uint32_t* r = v + 32 * h + 4 * g;
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                const int row = y + 16 * h + (lane >> 2) + 8 * k;
-                if (row < M && col < N) {
-                    const float2 val =
-                        make_float2(apply_alpha(r[2 * k], alpha), apply_alpha(r[2 * k + 1], alpha));
-                    *reinterpret_cast<float2*>(D + static_cast<int64_t>(row) * ldd + col) = val;
-                }
-            }
-        }
     }
 }
 
@@ -851,15 +803,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             uint32_t v[64];
             const uint32_t taddr = tmem_base + ACC_COL + (static_cast<uint32_t>(32 * q) << 16) +
                                    64 * chunk;
-            if (BF16) {
-                tmem_ld32(taddr, v);
-                tmem_ld32(taddr + 32, v + 32);
-            } else {
-                // two 16-lane halves; v[32h + 4g ..] = rows (lane / 4, lane / 4 + 8) of the
-                // half, columns 8g + 2 (lane % 4) and the next one
-                tmem_ld_16x256b_x8(taddr, v);
-                tmem_ld_16x256b_x8(taddr + (16u << 16), v + 32);
-            }
+            tmem_ld32(taddr, v);  // row `lane` of the quarter, columns [64 chunk, +64)
+            tmem_ld32(taddr + 32, v + 32);
             tmem_wait_ld();
             tc_fence_before();
             // this warp holds its slice: its arrival releases its part of the accumulator
@@ -871,11 +816,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             // first output row of this warp's slice: the CTA's half of the pair tile
             const int y = tm * PAIR_M + static_cast<int>(rank) * CTA_M + 32 * q;
             const int n0 = tn * BN + 64 * chunk;  // first output column
-            if (BF16)
-                store_slice<BF16, AMAX>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N,
-                                        &m_plain, &m_rht, flip);
-            else
-                store_f32_direct(v, alpha, static_cast<float*>(p.D), p.ldd, lane, n0, y, p.M, p.N);
+            store_slice<BF16, AMAX>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N, &m_plain,
+                                    &m_rht, flip);
         }
         if (lane == 0) bulk_wait_all();
         if (AMAX) {
@@ -967,8 +909,7 @@ bool make_scales_map(CUtensorMap* map, const uint8_t* scales, int64_t rows, int6
 }
 
 // 2D map over D (rows x N elements, row stride ldd) for the epilogue's bulk tensor stores
-// (the map clips rows beyond M): bf16 boxes of 32 rows x 16 bytes, unswizzled; FP32 boxes of
-// 32 rows x 64 bytes with the 64-byte swizzle.
+// (the map clips rows beyond M): boxes of 32 rows x 64 bytes with the 64-byte swizzle.
 bool make_output_map(CUtensorMap* map, void* D, int64_t M, int64_t N, int64_t ldd, bool bf16)
 {
     auto enc = tensor_map_encoder();
@@ -976,11 +917,11 @@ bool make_output_map(CUtensorMap* map, void* D, int64_t M, int64_t N, int64_t ld
     const int64_t esize = bf16 ? 2 : 4;
     const cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(ldd * esize)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>((bf16 ? 16 : 64) / esize), 32};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / esize), 32};
     const cuuint32_t estr[2] = {1, 1};
     return enc(map, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, D,
                dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-               bf16 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_64B,
+               CU_TENSOR_MAP_SWIZZLE_64B,
                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
