@@ -227,6 +227,23 @@ __device__ __forceinline__ float min3f(float a, float b, float c)
     return d;
 }
 
+__device__ __forceinline__ float max3f(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// Largest magnitude of v[0..n), n even, two values per three-input maximum (exact, any order).
+template <int N>
+__device__ __forceinline__ float absmax_f32(const float* v)
+{
+    float m = 0.0f;
+#pragma unroll
+    for (int j = 0; j < N; j += 2) m = max3f(m, fabsf(v[j]), fabsf(v[j + 1]));
+    return m;
+}
+
 // ---- paired FP32 lanes --------------------------------------------------------------------
 // sm_100 runs FP32 add, subtract, multiply and FMA on two lanes held in one 64-bit register
 // pair as one instruction (.f32x2).  Each lane is the IEEE operation with the stated rounding,

@@ -256,9 +256,7 @@ __global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
             const int64_t f = f0 + 32 * u;
             float e[8];
             unpack8(v[u], e);
-            float m = 0.0f;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(e[j]));
+            const float m = absmax_f32<8>(e);
             const float b = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
             const BlockScale bs = block_scale(b, ts.s_enc, r_tab);
             uint32_t packed = encode8<SR>(v[u], e, bs, philox, static_cast<uint64_t>(f), offset);
@@ -495,9 +493,7 @@ __global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR
             for (int q = 0; q < 4; ++q) {
                 float v[16];
                 load_row_block(q, v);
-                float m = 0.0f;
-#pragma unroll
-                for (int j = 0; j < 16; ++j) m = fmaxf(m, fabsf(v[j]));
+                const float m = absmax_f32<16>(v);
                 bmax[rrow][rblk + q] = m;
             }
             __syncthreads();
@@ -541,9 +537,7 @@ __global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR
                 if (BLOCK2D) {
                     b = tmax[rrow >> 4][rblk + q];
                 } else {
-                    b = 0.0f;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) b = fmaxf(b, fabsf(rv[j]));
+                    b = absmax_f32<16>(rv);
                 }
                 const BlockScale bs = block_scale(b, ts_row.s_enc, r_tab_row);
                 const uint64_t e0 = static_cast<uint64_t>(r) * a.cols + c0 + (rblk + q) * 16;
@@ -672,9 +666,7 @@ __global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR
                         if (BLOCK2D) {
                             b = tmax[2 * h + q][(2 * p + c) >> 4];
                         } else {
-                            b = 0.0f;
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(y[i]));
+                            b = absmax_f32<16>(y);
                         }
                         const BlockScale bs = block_scale(b, ts_col.s_enc, r_tab_col);
                         const uint64_t e0 =
