@@ -387,14 +387,15 @@ constexpr int tile_ctas_per_sm()
 }
 
 // Tile buffers per CTA.  Two (the next tile's copies in flight while this one is quantized),
-// except for the plain column-wise NVFP4 RTN passes (no RHT, no 16x16 scaling): they do little
-// arithmetic per byte, and one buffer halves their shared memory so that 8 CTAs share an SM,
-// which keeps more of HBM's latency covered (B200, 2^30 elements in rows of 4096: 0.976 ms
-// with one buffer and 8 CTAs against 1.10 ms with two buffers and 6).
+// except for the column-wise NVFP4 RTN passes without RHT (plain or 16x16-scaled): they do
+// little arithmetic per byte, and one buffer halves their shared memory so that 8 CTAs share an
+// SM, which keeps more of HBM's latency covered (B200: the plain column-wise pass on 2^30
+// elements in rows of 4096, 1.037 ms against 1.119 with two buffers and 6 CTAs; the 16x16
+// pass with both outputs on 8192 x 20480, 0.220 against 0.226 ms for the whole call).
 template <bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
 constexpr int tile_buffers()
 {
-    return COL && !BLOCK2D && !RHT && !SR && !MX ? 1 : 2;
+    return COL && !RHT && !SR && !MX ? 1 : 2;
 }
 template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
 constexpr int tile_min_ctas()
@@ -565,14 +566,14 @@ __global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR
 
         // Column walks.  Rows are a multiple of 64 whenever column-wise output is asked for, so
         // every tile has all 64 rows.
-        //  * The plain RTN pass (one buffer): thread t -> column t, all 64 rows (four blocks),
+        //  * The plain RTN pass: thread t -> column t, all 64 rows (four blocks),
         //    one 16-bit shared load per value; it writes 32 contiguous code bytes (a whole
         //    sector) and one scale word per output row.
         //  * Otherwise: thread t -> columns 2p, 2p + 1 (p = t % 64), rows 32h .. 32h + 31
         //    (h = t / 64); one 32-bit shared load brings a row's values of both columns.
         const int p = t & 63, h = t >> 6;
-        if (kBuffers == 1) {
-            if (COL && t < nc) {
+        if (COL && !BLOCK2D && !RHT && !SR && !MX) {
+            if (t < nc) {
                 const int64_t orow = c0 + t;  // output row = input column
                 uint32_t words[8];
                 uint32_t sfw = 0;
