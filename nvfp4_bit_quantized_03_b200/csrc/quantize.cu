@@ -280,16 +280,17 @@ __global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
 
 // ------------------------------------------------------------------------------------------
 // Pass 2b: tile quantizer.  A CTA stages 64-row x 128-column tiles in shared memory (rows
-// padded to 136 elements so that neither walk has bank conflicts), two buffers deep: while one
-// tile is quantized, the next one's rows are already being copied in (cp.async, 16 bytes per
-// copy, zero-filled outside the matrix).  Each tile gives
+// padded to 136 elements so that neither walk has bank conflicts) with cp.async (16 bytes per
+// copy, zero-filled outside the matrix), two buffers deep for most variants: while one tile is
+// quantized, the next one's rows are already being copied in (tile_buffers below).  Each tile
+// gives
 //   ROW: the row-wise output (blocks along the columns), thread t -> row t % 64, blocks
 //        4 (t / 64) .. +3: 32 contiguous code bytes and one scale word;
 //   COL: the column-wise output (x^T, blocks along the rows, optionally RHT'd), thread t ->
 //        the column pair 2 (t % 64), 2 (t % 64) + 1 and rows 32 (t / 64) .. +31 (two blocks):
 //        one 32-bit shared load brings a row's values of both columns, the Hadamard sign of
 //        that row flips both with one xor on the packed pair; per column 16 code bytes and two
-//        scale bytes.
+//        scale bytes.  The plain RTN pass walks one column per thread instead (in the kernel).
 // BLOCK2D: the scale of every 16x16 sub-tile comes from its maximum, shared by both outputs,
 // whose codes are then the same nibbles transposed.
 // ------------------------------------------------------------------------------------------
