@@ -486,6 +486,35 @@ def cpu_quantize_baseline(threads, log2n_1t=(20, 22, 24), log2n_all=(20, 22, 24,
             "single_thread": out["1t"], "all_cores": out["all"]}
 
 
+def cpu_gemm_baseline():
+    """The oracle's GEMM step timed alone: its plain FP64 triple loop (one thread) on the
+    fprop operands of the single-fprop workload (256 x 512 x 512) and of a 512-row slice of the
+    4096^3 layer, in GFLOP/s; numpy's FP64 BLAS on the same dequantized operands is timed too
+    and labelled "library"."""
+    import oracle
+    out = {"unit": "GFLOP/s", "kind": "oracle", "threads": 1, "blas_threads": blas_threads()}
+    for name, wl, rows in (("fprop_t256_i512_o512", synth.fprop_small(), None),
+                           ("linear_4096_first_512_rows", synth.layer_4096(), 512)):
+        lin = wl.linears[0]
+        X, W, _ = synth.linear_inputs(lin, wl.seed)
+        if rows is not None:
+            X = X[:rows]
+        qa, qb = oracle.fprop_operands(X, W)
+        A, B = qa.dequantize(), qb.dequantize()
+        flop = 2.0 * A.shape[0] * B.shape[0] * A.shape[1]
+        t0 = time.perf_counter()
+        oracle.gemm_ref_loop(A, B)
+        t_loop = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        for _ in range(5):
+            A @ B.T
+        t_blas = (time.perf_counter() - t0) / 5
+        out[name] = {"shape": f"{A.shape[0]} x {B.shape[0]} x {A.shape[1]}",
+                     "oracle_loop_gflops": flop / t_loop / 1e9,
+                     "library_numpy_fp64_gflops": flop / t_blas / 1e9}
+    return out
+
+
 def cpu_baseline(workload):
     threads = host_threads()
     secs, flops = oracle_sample(workload, tokens=1024, max_out=2048, max_in=5120,
@@ -497,7 +526,8 @@ def cpu_baseline(workload):
                       f"(C oracle, {threads} threads) + FP64 reference GEMMs (numpy matmul of "
                       "the dequantized operands)",
             "seconds": secs,
-            "quantize": cpu_quantize_baseline(threads)}
+            "quantize": cpu_quantize_baseline(threads),
+            "gemm": cpu_gemm_baseline()}
 
 
 def run_reference(args):
