@@ -624,7 +624,7 @@ def run_ours(args):
     e2e = None
     if not args.no_e2e:
         outs = step.output_host_buffers()
-        e2e_steps = max(1, min(args.steps, 5))
+        e2e_steps = max(1, min(args.steps, 10))
         barrier()
         torch.cuda.synchronize()
         s0 = torch.cuda.Event(enable_timing=True)
