@@ -300,7 +300,9 @@ __device__ __forceinline__ uint32_t rand16_as_f32_bits(uint32_t word, int h)
 }
 
 // Magnitude code of a >= 0 stochastically rounded with the random value whose FP32 pattern is
-// rbits = bits(2^23 + r16); the code is the low byte of the returned pattern.
+// rbits = bits(2^23 + r16); the code is the low byte of the returned pattern.  This is the
+// per-lane statement of the sequence; the quantizers run it two lanes at a time
+// (e2m1_sr_code2 below), with the same operations on each lane.
 __device__ __forceinline__ uint32_t e2m1_sr_code(float a, uint32_t rbits)
 {
     const float l0 = __fmaf_ru(a, 131072.0f, 8388608.0f);  // 2^23 + 2^17 a

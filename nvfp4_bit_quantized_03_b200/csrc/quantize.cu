@@ -381,7 +381,7 @@ __device__ __forceinline__ void rht16_presigned2(uint64_t* v)
 // CTAs per SM: the stochastic-rounding variants are bound by instruction issue and run fastest
 // with 4 CTAs of up to 128 registers (B200, 8192 x 20480: the one-pass SR pair 0.425 ms
 // against 0.452 with 5 CTAs and 0.476 with 6, where it spills), the RTN ones with 6 of 80.
-template <bool ROW, bool COL, bool SR>
+template <bool SR>
 constexpr int tile_ctas_per_sm()
 {
     return SR ? 4 : 6;
@@ -401,7 +401,7 @@ constexpr int tile_buffers()
 template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
 constexpr int tile_min_ctas()
 {
-    return tile_buffers<COL, BLOCK2D, RHT, SR, MX>() == 1 ? 8 : tile_ctas_per_sm<ROW, COL, SR>();
+    return tile_buffers<COL, BLOCK2D, RHT, SR, MX>() == 1 ? 8 : tile_ctas_per_sm<SR>();
 }
 
 template <bool ROW, bool COL, bool BLOCK2D, bool RHT, bool SR, bool MX>
