@@ -38,6 +38,8 @@ def _operands(M, N, K, seed=0, sr=False):
     (16, 16, 64),        # smallest shape
     (1024, 1536, 2048),  # many tiles, several k blocks per tile
     (384, 768, 4160),    # long K with a ragged last stage
+    (1344, 320, 512),    # more rows than columns: raster groups of 4 row tiles, a short last group
+    (20480, 528, 256),   # 240 pair tiles over the persistent grid, groups of 4, ragged N
 ])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_gemm_matches_oracle(M, N, K, dtype):
