@@ -75,8 +75,11 @@ typedef enum {
 /* Bits OR-ed into *dev_status by the kernels. */
 enum {
     NVFP4_DEVSTAT_NONFINITE = 1, /* a quantizer input (or its transform) held NaN/Inf     */
-    NVFP4_DEVSTAT_TIMEOUT = 2    /* a GEMM pipeline wait exceeded its time limit; the
+    NVFP4_DEVSTAT_TIMEOUT = 2,   /* a GEMM pipeline wait exceeded its time limit; the
                                     output of that GEMM is undefined                     */
+    NVFP4_DEVSTAT_BOUNDS = 4     /* (debug build only, see nvfp4_bounds_checked) a kernel
+                                    computed a global access outside its buffer and
+                                    skipped it; the outputs of that call are undefined   */
 };
 
 /* Quantizer flags. */
@@ -239,6 +242,28 @@ nvfp4_status nvfp4_gemm_amax(const nvfp4_operand* A, const nvfp4_operand* B, voi
  * waits end if a copy or an MMA never signals, without hanging the GPU.
  */
 nvfp4_status nvfp4_selftest_wait_timeout(int* dev_status, void* stream);
+
+/*
+ * Debug build (no counterpart on the pages).  The same sources compiled with
+ * -DNVFP4_BOUNDS_CHECK give libnvfp4_checked.so, with this header's API unchanged: every
+ * global load and store of the quantizers is checked against the extent of its buffer (the
+ * input's rows x ld values, the codes' rows x cols / 2 bytes, the scales' padded size), and
+ * every TMA box the GEMM issues against the TMA start rules (non-negative coordinates, a
+ * 16-byte aligned innermost start).  An access outside is skipped and NVFP4_DEVSTAT_BOUNDS is
+ * OR-ed into *dev_status; the call's outputs are then undefined.  Such a build is slower and
+ * meant for tests.
+ *
+ * nvfp4_bounds_checked returns 1 in that build and 0 in the normal one.
+ *
+ * nvfp4_selftest_bounds (checked build only; the normal one returns NVFP4_ERR_ARG and queues
+ * nothing): queues one kernel whose thread stores one word through the checked-store routine
+ * just past the end of a 16-byte buffer the routine is told about (the word itself lies inside
+ * a larger array the library owns, so nothing outside the library's memory is named).  The
+ * check refuses the store and sets NVFP4_DEVSTAT_BOUNDS in *dev_status (device, 4-byte
+ * aligned); the context stays usable.
+ */
+int nvfp4_bounds_checked(void);
+nvfp4_status nvfp4_selftest_bounds(int* dev_status, void* stream);
 
 /*
  * nvfp4_gemm for two MXFP4 operands (quantized with NVFP4_MX): the same tensor-core GEMM

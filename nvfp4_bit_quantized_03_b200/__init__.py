@@ -6,11 +6,13 @@ The Python surface is the ctypes binding in ``binding``; it loads the in-tree
 """
 from . import binding
 from .binding import (AMAX_GIVEN, BLOCK2D, COLWISE, OUT_BF16, OUT_F32, ROWWISE, SR,
-                      DEVSTAT_NONFINITE, DEVSTAT_TIMEOUT, NVFP4Error, QuantizedTensor, gemm,
+                      DEVSTAT_BOUNDS, DEVSTAT_NONFINITE, DEVSTAT_TIMEOUT, NVFP4Error,
+                      QuantizedTensor, bounds_checked, gemm,
                       linear_dgrad, linear_fprop, linear_wgrad, quantize, rht_quantize,
                       sign_mask_from_seed)
 
 __all__ = ["binding", "AMAX_GIVEN", "BLOCK2D", "COLWISE", "OUT_BF16", "OUT_F32", "ROWWISE", "SR",
-           "DEVSTAT_NONFINITE", "DEVSTAT_TIMEOUT", "NVFP4Error", "QuantizedTensor", "gemm",
+           "DEVSTAT_BOUNDS", "DEVSTAT_NONFINITE", "DEVSTAT_TIMEOUT", "NVFP4Error",
+           "QuantizedTensor", "bounds_checked", "gemm",
            "linear_dgrad", "linear_fprop", "linear_wgrad", "quantize", "rht_quantize",
            "sign_mask_from_seed"]

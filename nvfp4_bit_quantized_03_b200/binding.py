@@ -3,7 +3,11 @@
 Argument marshalling only: PyTorch owns the device memory and the streams; every step of the
 quantizers and GEMMs runs in the library's CUDA kernels.  There is no fallback: if the
 library is missing or a call fails, an exception is raised.
+
+Inside a ``with bounds_checked():`` block the same calls go to libnvfp4_checked.so, the debug
+build whose kernels check every global access against its buffer (NVFP4_DEVSTAT_BOUNDS).
 """
+import contextlib
 import ctypes
 import os
 import re
@@ -12,11 +16,12 @@ import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libnvfp4.so")
+CHECKED_LIB_PATH = os.path.join(_PKG, "libnvfp4_checked.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "nvfp4.h")
 
 # status codes and flags (include/nvfp4.h)
 OK, ERR_NULL, ERR_SHAPE, ERR_ALIGN, ERR_DEVICE, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_ARG = range(9)
-DEVSTAT_NONFINITE, DEVSTAT_TIMEOUT = 1, 2
+DEVSTAT_NONFINITE, DEVSTAT_TIMEOUT, DEVSTAT_BOUNDS = 1, 2, 4
 ROWWISE, COLWISE, BLOCK2D, SR, AMAX_GIVEN, MX = 1, 2, 4, 8, 16, 32
 OUT_F32, OUT_BF16 = 0, 1
 
@@ -32,7 +37,8 @@ class Operand(ctypes.Structure):
                 ("amax", ctypes.c_void_p), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64)]
 
 
-_lib = None
+_libs = {}               # path -> configured CDLL
+_active = LIB_PATH       # the library calls go to
 _poison = False
 
 
@@ -56,55 +62,76 @@ def _poisoned(t):
 
 
 def lib():
-    """Load libnvfp4.so (raises if it has not been built)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"libnvfp4.so not found at {LIB_PATH}; build it with "
-                              "`python -m nvfp4_bit_quantized_03_b200.build` (nvcc, sm_100a)")
-        L = ctypes.CDLL(LIB_PATH)
-        i64, u64, u16, vp, i32 = (ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint16,
-                                  ctypes.c_void_p, ctypes.c_int)
-        op = ctypes.POINTER(Operand)
-        sz = ctypes.c_size_t
-        L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
-        L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
-        L.nvfp4_codes_bytes.argtypes, L.nvfp4_codes_bytes.restype = [i64, i64], sz
-        L.nvfp4_scales_bytes.argtypes, L.nvfp4_scales_bytes.restype = [i64, i64], sz
-        L.nvfp4_workspace_bytes.argtypes = [i64, i64, ctypes.c_uint]
-        L.nvfp4_workspace_bytes.restype = sz
-        L.nvfp4_linear_workspace_bytes.argtypes = [i64, i64, i64]
-        L.nvfp4_linear_workspace_bytes.restype = sz
-        L.nvfp4_sign_mask_from_seed.argtypes, L.nvfp4_sign_mask_from_seed.restype = [u64], u16
-        L.nvfp4_scales_unswizzle.argtypes = [vp, i64, i64, vp]
-        L.nvfp4_scales_unswizzle.restype = i32
-        L.nvfp4_quantize.argtypes = [vp, i64, i64, i64, ctypes.c_uint, u64, u64, op, op, vp, vp, vp]
-        L.nvfp4_quantize.restype = i32
-        L.nvfp4_rht_quantize.argtypes = [vp, i64, i64, i64, u16, ctypes.c_uint, u64, u64, op, vp,
-                                         vp, vp]
-        L.nvfp4_rht_quantize.restype = i32
-        L.nvfp4_quantize_row_rht.argtypes = [vp, i64, i64, i64, u16, ctypes.c_uint, u64, u64, op,
-                                             op, vp, vp, vp]
-        L.nvfp4_quantize_row_rht.restype = i32
-        L.nvfp4_gemm.argtypes = [op, op, vp, i32, i64, vp, vp]
-        L.nvfp4_gemm.restype = i32
-        L.nvfp4_gemm_mx.argtypes = [op, op, vp, i32, i64, vp, vp]
-        L.nvfp4_gemm_mx.restype = i32
-        L.nvfp4_gemm_amax.argtypes = [op, op, vp, i64, u16, vp, vp, vp]
-        L.nvfp4_gemm_amax.restype = i32
-        L.nvfp4_selftest_wait_timeout.argtypes = [vp, vp]
-        L.nvfp4_selftest_wait_timeout.restype = i32
-        L.nvfp4_linear_fprop.argtypes = [vp, vp, i64, i64, i64, vp, i32, vp, vp, vp]
-        L.nvfp4_linear_fprop.restype = i32
-        L.nvfp4_linear_dgrad.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, i32, vp, vp, vp]
-        L.nvfp4_linear_dgrad.restype = i32
-        L.nvfp4_linear_wgrad.argtypes = [vp, vp, i64, i64, i64, u16, u64, u64, vp, i32, vp, vp, vp]
-        L.nvfp4_linear_wgrad.restype = i32
-        L.nvfp4_linear_dgrad_quantized.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, u16, u64,
-                                                   u64, op, op, vp, vp, vp]
-        L.nvfp4_linear_dgrad_quantized.restype = i32
-        _lib = L
-    return _lib
+    """The library calls go to: libnvfp4.so, or libnvfp4_checked.so inside bounds_checked()
+    (raises if it has not been built)."""
+    L = _libs.get(_active)
+    if L is None:
+        L = _libs[_active] = _open(_active)
+    return L
+
+
+@contextlib.contextmanager
+def bounds_checked():
+    """Route every call of this module made inside the block to libnvfp4_checked.so (the
+    -DNVFP4_BOUNDS_CHECK build: an out-of-extent global access is skipped and sets
+    NVFP4_DEVSTAT_BOUNDS in the call's status word).  Yields that library."""
+    global _active
+    prev = _active
+    _active = CHECKED_LIB_PATH
+    try:
+        yield lib()
+    finally:
+        _active = prev
+
+
+def _open(path):
+    if not os.path.exists(path):
+        raise ImportError(f"{os.path.basename(path)} not found at {path}; build it with "
+                          "`python -m nvfp4_bit_quantized_03_b200.build` (nvcc, sm_100a)")
+    L = ctypes.CDLL(path)
+    i64, u64, u16, vp, i32 = (ctypes.c_int64, ctypes.c_uint64, ctypes.c_uint16,
+                              ctypes.c_void_p, ctypes.c_int)
+    op = ctypes.POINTER(Operand)
+    sz = ctypes.c_size_t
+    L.nvfp4_version.argtypes, L.nvfp4_version.restype = [], i32
+    L.nvfp4_status_string.argtypes, L.nvfp4_status_string.restype = [i32], ctypes.c_char_p
+    L.nvfp4_codes_bytes.argtypes, L.nvfp4_codes_bytes.restype = [i64, i64], sz
+    L.nvfp4_scales_bytes.argtypes, L.nvfp4_scales_bytes.restype = [i64, i64], sz
+    L.nvfp4_workspace_bytes.argtypes = [i64, i64, ctypes.c_uint]
+    L.nvfp4_workspace_bytes.restype = sz
+    L.nvfp4_linear_workspace_bytes.argtypes = [i64, i64, i64]
+    L.nvfp4_linear_workspace_bytes.restype = sz
+    L.nvfp4_sign_mask_from_seed.argtypes, L.nvfp4_sign_mask_from_seed.restype = [u64], u16
+    L.nvfp4_scales_unswizzle.argtypes = [vp, i64, i64, vp]
+    L.nvfp4_scales_unswizzle.restype = i32
+    L.nvfp4_quantize.argtypes = [vp, i64, i64, i64, ctypes.c_uint, u64, u64, op, op, vp, vp, vp]
+    L.nvfp4_quantize.restype = i32
+    L.nvfp4_rht_quantize.argtypes = [vp, i64, i64, i64, u16, ctypes.c_uint, u64, u64, op, vp,
+                                     vp, vp]
+    L.nvfp4_rht_quantize.restype = i32
+    L.nvfp4_quantize_row_rht.argtypes = [vp, i64, i64, i64, u16, ctypes.c_uint, u64, u64, op,
+                                         op, vp, vp, vp]
+    L.nvfp4_quantize_row_rht.restype = i32
+    L.nvfp4_gemm.argtypes = [op, op, vp, i32, i64, vp, vp]
+    L.nvfp4_gemm.restype = i32
+    L.nvfp4_gemm_mx.argtypes = [op, op, vp, i32, i64, vp, vp]
+    L.nvfp4_gemm_mx.restype = i32
+    L.nvfp4_gemm_amax.argtypes = [op, op, vp, i64, u16, vp, vp, vp]
+    L.nvfp4_gemm_amax.restype = i32
+    L.nvfp4_selftest_wait_timeout.argtypes = [vp, vp]
+    L.nvfp4_selftest_wait_timeout.restype = i32
+    L.nvfp4_bounds_checked.argtypes, L.nvfp4_bounds_checked.restype = [], i32
+    L.nvfp4_selftest_bounds.argtypes, L.nvfp4_selftest_bounds.restype = [vp, vp], i32
+    L.nvfp4_linear_fprop.argtypes = [vp, vp, i64, i64, i64, vp, i32, vp, vp, vp]
+    L.nvfp4_linear_fprop.restype = i32
+    L.nvfp4_linear_dgrad.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, i32, vp, vp, vp]
+    L.nvfp4_linear_dgrad.restype = i32
+    L.nvfp4_linear_wgrad.argtypes = [vp, vp, i64, i64, i64, u16, u64, u64, vp, i32, vp, vp, vp]
+    L.nvfp4_linear_wgrad.restype = i32
+    L.nvfp4_linear_dgrad_quantized.argtypes = [vp, vp, i64, i64, i64, u64, u64, vp, u16, u64,
+                                               u64, op, op, vp, vp, vp]
+    L.nvfp4_linear_dgrad_quantized.restype = i32
+    return L
 
 
 def declared_functions():
@@ -295,6 +322,18 @@ def selftest_wait_timeout(dev_status, stream=None):
     status word has NVFP4_DEVSTAT_TIMEOUT set."""
     _check(lib().nvfp4_selftest_wait_timeout(_ptr(dev_status), _stream(stream)),
            "nvfp4_selftest_wait_timeout")
+
+
+def is_bounds_checked():
+    """nvfp4_bounds_checked of the library calls currently go to."""
+    return bool(lib().nvfp4_bounds_checked())
+
+
+def selftest_bounds(dev_status, stream=None):
+    """nvfp4_selftest_bounds (checked build only): one refused store past a buffer's declared
+    end; after it the device status word has NVFP4_DEVSTAT_BOUNDS set."""
+    _check(lib().nvfp4_selftest_bounds(_ptr(dev_status), _stream(stream)),
+           "nvfp4_selftest_bounds")
 
 
 def linear_fprop(X, W, out=None, out_dtype=torch.float32, workspace=None, dev_status=None,

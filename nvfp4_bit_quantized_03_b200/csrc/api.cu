@@ -168,7 +168,7 @@ nvfp4_status quantize_impl(const void* x, int64_t rows, int64_t cols, int64_t ld
         src.partials = static_cast<const uint32_t*>(workspace);
         src.n_partials = grid;
         st = from_cuda(launch_amax(xs, rows, cols, ld, rht, sign_mask,
-                                   static_cast<uint32_t*>(workspace), grid, s));
+                                   static_cast<uint32_t*>(workspace), grid, dev_status, s));
         if (st != NVFP4_OK) return st;
     }
     if (want_row && !want_col && !b2d && !mx) {
@@ -326,7 +326,7 @@ nvfp4_status nvfp4_quantize_row_rht(const void* x_bf16, int64_t rows, int64_t co
         src_row.partials = partials_plain;
         src_row.n_partials = grid;
         st = from_cuda(launch_amax_dual(xs, rows, cols, ld, sign_mask, partials_rht,
-                                        partials_plain, grid, s));
+                                        partials_plain, grid, dev_status, s));
         if (st != NVFP4_OK) return st;
     }
     TileArgs a{};
@@ -405,6 +405,26 @@ nvfp4_status nvfp4_selftest_wait_timeout(int* dev_status, void* stream)
     if (st != NVFP4_OK) return st;
     return from_cuda(launch_wait_selftest(dev_status, 50000000ull,  // 50 ms
                                           static_cast<cudaStream_t>(stream)));
+}
+
+int nvfp4_bounds_checked(void)
+{
+#ifdef NVFP4_BOUNDS_CHECK
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+nvfp4_status nvfp4_selftest_bounds(int* dev_status, void* stream)
+{
+    if (!nvfp4_bounds_checked()) return NVFP4_ERR_ARG;
+    if (!dev_status) return NVFP4_ERR_NULL;
+    if (!aligned4(dev_status)) return NVFP4_ERR_ALIGN;
+    int sms = 0;
+    const nvfp4_status st = current_device(&sms);
+    if (st != NVFP4_OK) return st;
+    return from_cuda(launch_bounds_selftest(dev_status, static_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_gemm_mx(const nvfp4_operand* A, const nvfp4_operand* B, void* D, int d_dtype,

@@ -49,6 +49,7 @@
 #include <cstdint>
 #include <mutex>
 
+#include "bounds_check.cuh"
 #include "nvfp4_internal.h"
 
 namespace nvfp4 {
@@ -294,6 +295,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
 }
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Debug builds (bounds_check.cuh): a tiled TMA box must start at non-negative coordinates with
+// its innermost coordinate on a 16-byte boundary (x * element bytes); a start beyond the far
+// edge is legal (loads zero-fill, stores are clipped).  Records NVFP4_DEVSTAT_BOUNDS otherwise.
+__device__ __forceinline__ bool tma_box_start_ok(int x, int y, int elem_bytes, int* dev_status)
+{
+    if (x >= 0 && y >= 0 && (x * elem_bytes) % 16 == 0) return true;
+    record_bounds_error(dev_status);
+    return false;
+}
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---- tcgen05 -----------------------------------------------------------------------------
@@ -466,7 +477,8 @@ template <bool BF16, bool AMAX = false>
 __device__ __forceinline__ void store_slice(const uint32_t* v, const Alpha& alpha, uint32_t stage_buf,
                                             int lane, const CUtensorMap* tmap_d, int n0, int y,
                                             int M, int N, uint32_t* m_plain = nullptr,
-                                            uint32_t* m_rht = nullptr, uint32_t flip = 0)
+                                            uint32_t* m_rht = nullptr, uint32_t flip = 0,
+                                            int* dev_status = nullptr)
 {
     constexpr int CHUNKS = 4;                        // 16-byte chunks per box row
     constexpr int COLS = CHUNKS * (BF16 ? 8 : 4);    // columns per box row
@@ -520,7 +532,9 @@ __device__ __forceinline__ void store_slice(const uint32_t* v, const Alpha& alph
         fence_async_smem();
         __syncwarp();
         const int x = n0 + r * COLS;
-        if (lane == 0 && y < M && x < N) tma_store_2d(tmap_d, stage_buf, x, y);
+        if (lane == 0 && y < M && x < N &&
+            (!kBoundsCheck || tma_box_start_ok(x, y, BF16 ? 2 : 4, dev_status)))
+            tma_store_2d(tmap_d, stage_buf, x, y);
     }
 }
 
@@ -604,6 +618,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int ga = tm * 2 + static_cast<int>(rank);  // this CTA's 128-row group of A
             for (int kb = 0; kb < num_kb; ++kb) {
                 if (!wait_bounded(bar(BAR_EMPTY + stage), phase ^ 1, abort_flag, p.dev_status)) {
+                    ok = false;
+                    break;
+                }
+                if (kBoundsCheck &&
+                    !(tma_box_start_ok(kb * (BK / 2), ga * CTA_M, 1, p.dev_status) &&
+                      kb * (BK / 2) < p.K / 2 &&
+                      tma_box_start_ok(kb * (BK / 2), tn * BN + static_cast<int>(rank) * B_ROWS, 1,
+                                       p.dev_status))) {
+                    // no copy for this stage: the roles waiting for it stop at the abort flag
+                    record_bounds_error(p.dev_status);
+                    *abort_flag = 1;
                     ok = false;
                     break;
                 }
@@ -822,7 +847,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             const int y = tm * PAIR_M + static_cast<int>(rank) * CTA_M + 32 * q;
             const int n0 = tn * BN + 64 * chunk;  // first output column
             store_slice<BF16, AMAX>(v, alpha, stage_buf, lane, &tmap_d, n0, y, p.M, p.N, &m_plain,
-                                    &m_rht, flip);
+                                    &m_rht, flip, p.dev_status);
         }
         if (lane == 0) bulk_wait_all();
         if (AMAX) {

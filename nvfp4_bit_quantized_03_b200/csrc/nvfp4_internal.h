@@ -57,18 +57,23 @@ struct TileArgs {
 
 int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count);
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool rht,
-                        uint32_t sign_mask, uint32_t* partials, int grid, cudaStream_t s);
+                        uint32_t sign_mask, uint32_t* partials, int grid, int* dev_status,
+                        cudaStream_t s);
 // One pass for both maxima of the dual mode: amax of RHT(x) along the rows into
 // `partials_rht` and amax of x into `partials_plain` (grid entries each).
 cudaError_t launch_amax_dual(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                              uint32_t sign_mask, uint32_t* partials_rht,
-                             uint32_t* partials_plain, int grid, cudaStream_t s);
+                             uint32_t* partials_plain, int grid, int* dev_status,
+                             cudaStream_t s);
 cudaError_t launch_quant_rowwise(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                                  const QuantSource& src, float* amax_out0, float* amax_out1,
                                  uint8_t* codes, uint8_t* scales, bool sr, uint64_t seed,
                                  uint64_t offset, int* dev_status, int sm_count, cudaStream_t s);
 cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2d, bool rht,
                               bool sr, bool mx, int sm_count, cudaStream_t s);
+// Debug build only: one checked store just past a buffer's declared end (refused, recorded as
+// NVFP4_DEVSTAT_BOUNDS); cudaErrorNotSupported in the normal build.
+cudaError_t launch_bounds_selftest(int* dev_status, cudaStream_t s);
 
 struct GemmArgs {
     const uint8_t* a_codes;

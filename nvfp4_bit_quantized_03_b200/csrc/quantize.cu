@@ -23,6 +23,7 @@
 
 #include <cstdint>
 
+#include "bounds_check.cuh"
 #include "nvfp4_device.cuh"
 #include "nvfp4_internal.h"
 
@@ -34,8 +35,10 @@ namespace nvfp4 {
 
 __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t rows,
                                                    int64_t cols, int64_t ld,
-                                                   uint32_t* __restrict__ partials)
+                                                   uint32_t* __restrict__ partials,
+                                                   int* dev_status)
 {
+    const int64_t xb = bf16_matrix_bytes(rows, cols, ld);  // extent of x (bounds checks)
     const int64_t cpr = cols >> 3;  // 16-byte chunks per row
     const int64_t total = rows * cpr;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -44,16 +47,19 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
     if (ld == cols) {
         const uint4* p = reinterpret_cast<const uint4*>(x);
         for (; i + 3 * stride < total; i += 4 * stride) {
-            const uint4 a = __ldg(p + i), b = __ldg(p + i + stride);
-            const uint4 c = __ldg(p + i + 2 * stride), d = __ldg(p + i + 3 * stride);
+            const uint4 a = ldg_checked(p + i, x, xb, dev_status);
+            const uint4 b = ldg_checked(p + i + stride, x, xb, dev_status);
+            const uint4 c = ldg_checked(p + i + 2 * stride, x, xb, dev_status);
+            const uint4 d = ldg_checked(p + i + 3 * stride, x, xb, dev_status);
             m = max(m, max(max(absmax_bits8(a), absmax_bits8(b)),
                            max(absmax_bits8(c), absmax_bits8(d))));
         }
-        for (; i < total; i += stride) m = max(m, absmax_bits8(__ldg(p + i)));
+        for (; i < total; i += stride) m = max(m, absmax_bits8(ldg_checked(p + i, x, xb, dev_status)));
     } else {
         for (; i < total; i += stride) {
             const int64_t r = i / cpr, c = i - r * cpr;
-            m = max(m, absmax_bits8(__ldg(reinterpret_cast<const uint4*>(x + r * ld) + c)));
+            m = max(m, absmax_bits8(ldg_checked(reinterpret_cast<const uint4*>(x + r * ld) + c,
+                                                x, xb, dev_status)));
         }
     }
     block_max_store(m, partials + blockIdx.x);
@@ -67,7 +73,8 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
                                                        int64_t rows, int64_t cols, int64_t ld,
                                                        uint32_t sign_mask,
                                                        uint32_t* __restrict__ partials,
-                                                       uint32_t* __restrict__ partials_plain)
+                                                       uint32_t* __restrict__ partials_plain,
+                                                       int* dev_status)
 {
     // The transform's sign flips are applied to the packed bf16 pairs (one xor per two
     // values), and its final x1/4 is applied once to the maximum: rounding is monotone, so the
@@ -76,6 +83,7 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
 #pragma unroll
     for (int k = 0; k < 16; ++k) flip[k] = ((sign_mask >> k) & 1u) ? 0x80008000u : 0u;
     uint32_t mp = 0;
+    const int64_t xb = bf16_matrix_bytes(rows, cols, ld);  // extent of x (bounds checks)
     const int64_t cpr = cols >> 2;  // 8-byte column groups per row
     const int64_t total = (rows >> 4) * cpr;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
@@ -86,7 +94,8 @@ __global__ void __launch_bounds__(256) amax_rht_kernel(const uint16_t* __restric
         const uint16_t* base = x + (g << 4) * ld + (c << 2);
         uint2 v[16];
 #pragma unroll
-        for (int k = 0; k < 16; ++k) v[k] = __ldg(reinterpret_cast<const uint2*>(base + k * ld));
+        for (int k = 0; k < 16; ++k)
+            v[k] = ldg_checked(reinterpret_cast<const uint2*>(base + k * ld), x, xb, dev_status);
         if (PLAIN) {
 #pragma unroll
             for (int k = 0; k < 16; ++k)
@@ -163,14 +172,17 @@ __device__ __forceinline__ TensorScale fold_amax(const QuantSource& src, float* 
 
 // Zero the scale words of the padding rows [rows, rows_pad) of a scale buffer.
 __device__ __forceinline__ void zero_scale_padding(uint8_t* scales, int64_t rows, int64_t cols,
-                                                   int64_t first_item, int64_t item_stride)
+                                                   int64_t first_item, int64_t item_stride,
+                                                   int* dev_status)
 {
+    const int64_t sb = scales_extent(rows, cols);
     const int64_t gpr = cols >> 6;  // 4-block groups per row
     const int64_t rows_pad = (rows + 127) & ~static_cast<int64_t>(127);
     const int64_t n = (rows_pad - rows) * gpr;
     for (int64_t i = first_item; i < n; i += item_stride) {
         const int64_t r = rows + i / gpr, g = i % gpr;
-        *reinterpret_cast<uint32_t*>(scales + sf_offset(r, g << 2, gpr)) = 0u;
+        st_checked(reinterpret_cast<uint32_t*>(scales + sf_offset(r, g << 2, gpr)), 0u, scales, sb,
+                   dev_status);
     }
 }
 
@@ -217,6 +229,9 @@ __global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
     const int64_t wstride = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
     const int64_t wfirst = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const bool contiguous = ld == cols;
+    // buffer extents (bounds checks)
+    const int64_t xb = bf16_matrix_bytes(rows, cols, ld);
+    const int64_t cb = codes_extent(rows, cols), sb = scales_extent(rows, cols);
 
     // Row and column of this lane's first chunk, kept up to date without dividing: each
     // iteration moves back by D = wstride * 128 chunks = dq rows and dr chunks.
@@ -236,8 +251,9 @@ __global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
                 const int64_t f = f0 + 32 * u;
                 v[u] = make_uint4(0, 0, 0, 0);
                 if (f < total)
-                    v[u] = __ldg(contiguous ? reinterpret_cast<const uint4*>(x) + f
-                                            : reinterpret_cast<const uint4*>(x + ru * ld) + cu);
+                    v[u] = ldg_checked(contiguous ? reinterpret_cast<const uint4*>(x) + f
+                                                  : reinterpret_cast<const uint4*>(x + ru * ld) + cu,
+                                       x, xb, dev_status);
                 cu += 32;
                 while (cu >= cpr) {
                     cu -= cpr;
@@ -266,16 +282,16 @@ __global__ void __launch_bounds__(256, 3) quant_rowwise_kernel(
             const uint32_t s2 = __shfl_down_sync(0xFFFFFFFFu, sf, 4);
             const uint32_t s3 = __shfl_down_sync(0xFFFFFFFFu, sf, 6);
             if (f < total) {
-                reinterpret_cast<uint32_t*>(codes)[f] = packed;
+                st_checked(reinterpret_cast<uint32_t*>(codes) + f, packed, codes, cb, dev_status);
                 if ((lane & 7) == 0)
-                    *reinterpret_cast<uint32_t*>(scales + sf_offset(rr[u], cc[u] >> 1, gpr)) =
-                        sf | (s1 << 8) | (s2 << 16) | (s3 << 24);
+                    st_checked(reinterpret_cast<uint32_t*>(scales + sf_offset(rr[u], cc[u] >> 1, gpr)),
+                               sf | (s1 << 8) | (s2 << 16) | (s3 << 24), scales, sb, dev_status);
             }
         }
     }
     zero_scale_padding(scales, rows, cols,
                        static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x,
-                       static_cast<int64_t>(gridDim.x) * blockDim.x);
+                       static_cast<int64_t>(gridDim.x) * blockDim.x, dev_status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -332,8 +348,14 @@ __device__ __forceinline__ void tile_load_async(const TileArgs& a, uint16_t* buf
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
         const int ch = t + 128 * k, row = ch >> 4, cc = ch & 15;
-        const bool in = row < nr && cc * 8 < nc;
+        bool in = row < nr && cc * 8 < nc;
         const uint16_t* src = in ? a.x + (r0 + row) * a.ld + c0 + cc * 8 : a.x;
+        if (kBoundsCheck && in &&
+            !in_buffer(reinterpret_cast<const uint4*>(src), a.x,
+                       bf16_matrix_bytes(a.rows, a.cols, a.ld), a.dev_status)) {
+            in = false;  // zero-filled instead
+            src = a.x;
+        }
         const uint32_t dst = base + 2u * static_cast<uint32_t>(row * kTilePitch + cc * 8);
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                      "r"(in ? 16 : 0)
@@ -559,10 +581,14 @@ __global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR
                 for (int q = 0; q < 8; ++q) words[q] = 0;
             }
             uint4* dst = reinterpret_cast<uint4*>(a.row_codes + (r * a.cols + c0 + rblk * 16) / 2);
-            dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-            dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-            *reinterpret_cast<uint32_t*>(a.row_scales +
-                                         sf_offset(r, (c0 >> 4) + rblk, a.cols >> 6)) = sfw;
+            const int64_t cb = codes_extent(a.rows, a.cols), sb = scales_extent(a.rows, a.cols);
+            st_checked(dst, make_uint4(words[0], words[1], words[2], words[3]), a.row_codes, cb,
+                       a.dev_status);
+            st_checked(dst + 1, make_uint4(words[4], words[5], words[6], words[7]), a.row_codes,
+                       cb, a.dev_status);
+            st_checked(reinterpret_cast<uint32_t*>(a.row_scales +
+                                                   sf_offset(r, (c0 >> 4) + rblk, a.cols >> 6)),
+                       sfw, a.row_scales, sb, a.dev_status);
         }
 
         // Column walks.  Rows are a multiple of 64 whenever column-wise output is asked for, so
@@ -598,10 +624,14 @@ __global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR
                     for (int q = 0; q < 8; ++q) words[q] = 0;
                 }
                 uint4* dst = reinterpret_cast<uint4*>(a.col_codes + (orow * a.rows + r0) / 2);
-                dst[0] = make_uint4(words[0], words[1], words[2], words[3]);
-                dst[1] = make_uint4(words[4], words[5], words[6], words[7]);
-                *reinterpret_cast<uint32_t*>(a.col_scales +
-                                             sf_offset(orow, r0 >> 4, a.rows >> 6)) = sfw;
+                const int64_t cb = codes_extent(a.cols, a.rows), sb = scales_extent(a.cols, a.rows);
+                st_checked(dst, make_uint4(words[0], words[1], words[2], words[3]), a.col_codes,
+                           cb, a.dev_status);
+                st_checked(dst + 1, make_uint4(words[4], words[5], words[6], words[7]),
+                           a.col_codes, cb, a.dev_status);
+                st_checked(reinterpret_cast<uint32_t*>(a.col_scales +
+                                                       sf_offset(orow, r0 >> 4, a.rows >> 6)),
+                           sfw, a.col_scales, sb, a.dev_status);
             }
         } else if (COL && 2 * p < nc) {
             const uint32_t* tile32 = reinterpret_cast<const uint32_t*>(tile) + p;
@@ -692,19 +722,21 @@ __global__ void __launch_bounds__(128, (tile_min_ctas<ROW, COL, BLOCK2D, RHT, SR
                     for (int q = 0; q < 4; ++q) words[c][q] = 0;
                 }
                 const int64_t orow = c0 + 2 * p + c;  // output row = input column
-                *reinterpret_cast<uint4*>(a.col_codes + (orow * a.rows + r0 + 32 * h) / 2) =
-                    make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]);
-                *reinterpret_cast<uint16_t*>(
-                    a.col_scales + sf_offset(orow, (r0 >> 4) + 2 * h, a.rows >> 6)) =
-                    static_cast<uint16_t>(sfw[c]);
+                st_checked(reinterpret_cast<uint4*>(a.col_codes + (orow * a.rows + r0 + 32 * h) / 2),
+                           make_uint4(words[c][0], words[c][1], words[c][2], words[c][3]),
+                           a.col_codes, codes_extent(a.cols, a.rows), a.dev_status);
+                st_checked(reinterpret_cast<uint16_t*>(
+                               a.col_scales + sf_offset(orow, (r0 >> 4) + 2 * h, a.rows >> 6)),
+                           static_cast<uint16_t>(sfw[c]), a.col_scales,
+                           scales_extent(a.cols, a.rows), a.dev_status);
             }
         }
         __syncthreads();  // everyone is done with this buffer before it is refilled
     }
     const int64_t first = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
-    if (ROW) zero_scale_padding(a.row_scales, a.rows, a.cols, first, step);
-    if (COL) zero_scale_padding(a.col_scales, a.cols, a.rows, first, step);
+    if (ROW) zero_scale_padding(a.row_scales, a.rows, a.cols, first, step, a.dev_status);
+    if (COL) zero_scale_padding(a.col_scales, a.cols, a.rows, first, step, a.dev_status);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -742,22 +774,24 @@ int amax_grid(int64_t rows, int64_t cols, bool rht, int sm_count)
 }
 
 cudaError_t launch_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld, bool rht,
-                        uint32_t sign_mask, uint32_t* partials, int grid, cudaStream_t s)
+                        uint32_t sign_mask, uint32_t* partials, int grid, int* dev_status,
+                        cudaStream_t s)
 {
     if (rht)
         amax_rht_kernel<false><<<grid, 256, 0, s>>>(x, rows, cols, ld, sign_mask, partials,
-                                                     nullptr);
+                                                     nullptr, dev_status);
     else
-        amax_kernel<<<grid, 256, 0, s>>>(x, rows, cols, ld, partials);
+        amax_kernel<<<grid, 256, 0, s>>>(x, rows, cols, ld, partials, dev_status);
     return cudaGetLastError();
 }
 
 cudaError_t launch_amax_dual(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld,
                              uint32_t sign_mask, uint32_t* partials_rht,
-                             uint32_t* partials_plain, int grid, cudaStream_t s)
+                             uint32_t* partials_plain, int grid, int* dev_status,
+                             cudaStream_t s)
 {
     amax_rht_kernel<true><<<grid, 256, 0, s>>>(x, rows, cols, ld, sign_mask, partials_rht,
-                                                partials_plain);
+                                                partials_plain, dev_status);
     return cudaGetLastError();
 }
 
@@ -833,6 +867,31 @@ cudaError_t launch_quant_tile(const TileArgs& a, bool row, bool col, bool block2
     else if (col && !rht && !sr)          launch_tile_t<false, true, false, false, false>(a, g, sm, s);
     else return cudaErrorInvalidValue;
     return cudaGetLastError();
+}
+
+#ifdef NVFP4_BOUNDS_CHECK
+// The self-test's array: 32 bytes, of which the check is told about the first 16.
+__device__ uint32_t g_bounds_probe[8];
+
+__global__ void bounds_selftest_kernel(int* dev_status)
+{
+    // word 3 is inside the declared 16 bytes and is written; word 4 is the first past them and
+    // is refused (it is still inside the array, so even an unchecked store would stay there)
+    st_checked(g_bounds_probe + 3, 1u, g_bounds_probe, 16, dev_status);
+    st_checked(g_bounds_probe + 4, 1u, g_bounds_probe, 16, dev_status);
+}
+#endif
+
+cudaError_t launch_bounds_selftest(int* dev_status, cudaStream_t s)
+{
+#ifdef NVFP4_BOUNDS_CHECK
+    bounds_selftest_kernel<<<1, 1, 0, s>>>(dev_status);
+    return cudaGetLastError();
+#else
+    (void)dev_status;
+    (void)s;
+    return cudaErrorNotSupported;
+#endif
 }
 
 }  // namespace nvfp4

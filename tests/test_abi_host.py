@@ -1,6 +1,7 @@
 """Host-side checks of the C ABI that need no GPU: the library loads, exports every function
 include/nvfp4.h declares, sizes its buffers as documented, and rejects invalid arguments
 before queueing any work."""
+import contextlib
 import ctypes
 
 import numpy as np
@@ -244,3 +245,39 @@ def test_binding_rejects_bad_output_tensors_before_calling():
 def test_wait_selftest_rejects_a_null_status_word():
     # argument checks come before any device access
     assert B.lib().nvfp4_selftest_wait_timeout(None, None) == B.ERR_NULL
+
+
+def test_checked_build_exports_the_same_functions_and_says_it_is_checked():
+    names = B.declared_functions()
+    assert "nvfp4_bounds_checked" in names and "nvfp4_selftest_bounds" in names
+    assert B.lib().nvfp4_bounds_checked() == 0
+    with B.bounds_checked() as L:
+        assert L is B.lib()
+        missing = [n for n in names if not hasattr(L, n)]
+        assert not missing, missing
+        assert L.nvfp4_bounds_checked() == 1
+        assert B.is_bounds_checked()
+    # the block routes calls only while it is open
+    assert not B.is_bounds_checked()
+
+
+def test_bounds_selftest_argument_checks():
+    # the normal build refuses before any device access; the checked build checks the
+    # status word before any device access
+    assert B.lib().nvfp4_selftest_bounds(ctypes.c_void_p(0x1000), None) == B.ERR_ARG
+    with B.bounds_checked() as L:
+        assert L.nvfp4_selftest_bounds(None, None) == B.ERR_NULL
+        assert L.nvfp4_selftest_bounds(ctypes.c_void_p(0x1002), None) == B.ERR_ALIGN
+
+
+def test_checked_build_rejects_invalid_arguments_like_the_normal_one():
+    out = _op(256, 512)
+    for lib_ctx in (contextlib.nullcontext(B.lib()), B.bounds_checked()):
+        with lib_ctx as L:
+            # cols not a multiple of 64, and a flag combination the API refuses
+            assert L.nvfp4_quantize(ctypes.c_void_p(0x1000), 256, 520, 520, B.ROWWISE, 0, 0,
+                                    ctypes.byref(out), None, ctypes.c_void_p(0x8000), None,
+                                    None) == B.ERR_SHAPE
+            assert L.nvfp4_quantize(ctypes.c_void_p(0x1000), 256, 512, 512,
+                                    B.BLOCK2D | B.SR | B.ROWWISE, 0, 0, ctypes.byref(out), None,
+                                    ctypes.c_void_p(0x8000), None, None) == B.ERR_ARG
