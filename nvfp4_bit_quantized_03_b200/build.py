@@ -47,6 +47,7 @@ def _sources():
         if name.endswith((".cu", ".cuh", ".h")):
             out.append(os.path.join(CSRC, name))
     out.append(os.path.join(INCLUDE, "nvfp4.h"))
+    out.append(os.path.abspath(__file__))  # a change of flags rebuilds too
     return out
 
 

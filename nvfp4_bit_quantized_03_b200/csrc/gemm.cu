@@ -33,9 +33,9 @@
 //               CTA's 128 x 256 half of the accumulator (tcgen05.ld), releases it to the leader,
 //               scales by 1 / (S_enc,A S_enc,B) and writes it while the next tile computes,
 //               through a 2 KB per-warp staging buffer with TMA bulk tensor stores (2 rounds for
-//               bf16, 4 for FP32; clipped at the matrix edge).  With
-//               the fused amax, the bf16 epilogue also reduces max |D| and, by 16-lane shuffles
-//               across rows, max |RHT(D)| for the next quantization of D.
+//               bf16, 4 for FP32; clipped at the matrix edge).  With the fused amax, the bf16
+//               epilogue also reduces max |D| and, by 16-lane shuffles across rows,
+//               max |RHT(D)| for the next quantization of D.
 // No load is multicast: every CTA loads its own operands from this GPU's memory.
 // Every wait on an mbarrier is bounded in time; on expiry the kernel records
 // NVFP4_DEVSTAT_TIMEOUT, drains its in-flight copies and MMAs (again with a limit), meets its
