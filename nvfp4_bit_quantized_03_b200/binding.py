@@ -74,7 +74,8 @@ def lib():
 def bounds_checked():
     """Route every call of this module made inside the block to libnvfp4_checked.so (the
     -DNVFP4_BOUNDS_CHECK build: an out-of-extent global access is skipped and sets
-    NVFP4_DEVSTAT_BOUNDS in the call's status word).  Yields that library."""
+    NVFP4_DEVSTAT_BOUNDS in the call's status word).  Yields that library.  The switch is
+    process-wide, not per thread: other threads' calls inside the block go there too."""
     global _active
     prev = _active
     _active = CHECKED_LIB_PATH
