@@ -35,17 +35,22 @@ FP4_OVER_BF16 = 4.0  # nominal dense FP4 : BF16 tensor throughput on B200 (9 : 2
 GEMM_BF16_DRAM_BYTES = 394.2e6
 
 
-def _peaks():
-    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+def _peaks(path=None):
+    """The roofline denominators: the measured copy bandwidth and bf16 GEMM rates of this
+    machine's GPUs when MEASURED_PEAKS.json holds them as numbers, else the fallback figures."""
+    path = path or os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
-        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
-                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
-                "source": "measured"}
-    except (OSError, KeyError, ValueError):
-        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-                "source": "fallback"}
+        out = {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+               "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+               "source": "measured"}
+        if all(v > 0 for k, v in out.items() if k != "source"):
+            return out
+    except (OSError, KeyError, ValueError, TypeError, AttributeError):
+        pass
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
 
 
 # ---- multi-rank plumbing (also exercised by the CPU gloo tests) --------------------------

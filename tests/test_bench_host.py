@@ -70,3 +70,24 @@ def test_reference_arm_nonzero_rank_exits_quietly():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
                           "--steps", "1"], capture_output=True, text=True, env=env, timeout=120)
     assert out.returncode == 0 and out.stdout.strip() == ""
+
+
+def test_peaks_read_the_measured_file_and_fall_back_on_anything_else(tmp_path):
+    good = tmp_path / "good.json"
+    good.write_text(json.dumps({"hbm_gbs": 7100.5, "bf16_tflops": 1650, "bf16_tflops_sustained":
+                                1420, "clocks": {"sm": 1965}}))
+    p = bench._peaks(str(good))
+    assert p["source"] == "measured" and p["hbm_gbs"] == 7100.5
+    assert p["bf16_tflops"] == 1650.0 and p["bf16_tflops_sustained"] == 1420.0
+    no_sustained = tmp_path / "burst_only.json"
+    no_sustained.write_text(json.dumps({"hbm_gbs": 7000, "bf16_tflops": 1600}))
+    assert bench._peaks(str(no_sustained))["bf16_tflops_sustained"] == 1600.0
+    for i, bad in enumerate(['{"hbm_gbs": {"value": 7000}, "bf16_tflops": 1600}',
+                             '{"hbm_gbs": "n/a", "bf16_tflops": 1600}',
+                             '{"hbm_gbs": 0, "bf16_tflops": 1600}',
+                             '{"bf16_tflops": 1600}', '[1, 2]', 'not json']):
+        f = tmp_path / f"bad{i}.json"
+        f.write_text(bad)
+        p = bench._peaks(str(f))
+        assert p["source"] == "fallback" and p["hbm_gbs"] == 6650.0, bad
+    assert bench._peaks(str(tmp_path / "missing.json"))["source"] == "fallback"
